@@ -1,1 +1,13 @@
-"""B200-native exact attention forward (placeholder; binding added with the kernel)."""
+"""Exact attention forward for B200 (sm_100a): one fused tcgen05/TMA kernel
+behind a C ABI (include/attn_fwd.h), with this thin Python binding.
+
+    o, lse = attn_fwd(q, k, v, causal=True)
+
+computes O = softmax(scale*QK^T [+causal mask]) V and the per-row natural-log
+log-sum-exp, for bf16 [B, H, N, d] CUDA tensors with d in {64, 128}.
+"""
+from ._lib import (AttnError, attn_fwd, attn_fwd_host, device_status, header_functions,
+                   host_workspace_bytes, load_library, status_str, version)
+
+__all__ = ["AttnError", "attn_fwd", "attn_fwd_host", "device_status", "header_functions",
+           "host_workspace_bytes", "load_library", "status_str", "version"]

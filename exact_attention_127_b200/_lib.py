@@ -1,0 +1,183 @@
+"""ctypes binding of libattn127.so: argument marshalling only.
+
+Every step of the attention computation runs in the library's CUDA kernel;
+this module only checks tensor metadata, allocates outputs through PyTorch and
+forwards pointers.  There is no fallback: if the library is missing, or the
+device is not an sm_100 GPU, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+import torch
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libattn127.so")
+HEADER_PATH = os.path.join(os.path.dirname(PKG), "include", "attn_fwd.h")
+
+ATTN_OK = 0
+
+
+class AttnError(RuntimeError):
+    """A non-zero status returned by the C library."""
+
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_str(status)} (status {status})")
+
+
+_lib = None
+
+
+def load_library():
+    """Load (once) and return the ctypes handle of libattn127.so."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"CUDA library {LIB_PATH} is missing; build it with "
+            "`python -m exact_attention_127_b200.build` (there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i64, c_int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, c_int, ctypes.c_float, vp]
+    lib.attn_fwd.restype = c_int
+    lib.attn_fwd_host.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, c_int, ctypes.c_float,
+                                  vp, ctypes.c_size_t, vp]
+    lib.attn_fwd_host.restype = c_int
+    lib.attn_fwd_host_workspace_bytes.argtypes = [i64, i64, i64, i64]
+    lib.attn_fwd_host_workspace_bytes.restype = ctypes.c_size_t
+    lib.attn_device_status.argtypes = [vp, c_int]
+    lib.attn_device_status.restype = c_int
+    lib.attn_status_str.argtypes = [c_int]
+    lib.attn_status_str.restype = ctypes.c_char_p
+    lib.attn_version.argtypes = []
+    lib.attn_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def header_functions(path: str = HEADER_PATH):
+    """Names of the functions the public header declares."""
+    text = open(path).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_\w+)\s*\(", text)))
+
+
+def status_str(status: int) -> str:
+    return load_library().attn_status_str(int(status)).decode()
+
+
+def version() -> str:
+    return load_library().attn_version().decode()
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check_inputs(q, k, v, device_expected: bool):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+        if t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be bfloat16, got {t.dtype}")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be [B, H, N, d], got shape {tuple(t.shape)}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if device_expected and not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not device_expected and t.is_cuda:
+            raise ValueError(f"{name} must be a CPU tensor")
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k, v must share one [B, H, N, d] shape")
+    if device_expected and not (q.device == k.device == v.device):
+        raise ValueError("q, k, v must be on one device")
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+             scale: float | None = None, out: torch.Tensor | None = None,
+             lse: torch.Tensor | None = None, stream=None):
+    """O = softmax(scale*QK^T [+causal mask]) V and LSE, on the GPU.
+
+    q, k, v: bf16 CUDA tensors [B, H, N, d], contiguous, d in {64, 128}.
+    Returns (o bf16 [B, H, N, d], lse fp32 [B, H, N]).  Asynchronous on
+    `stream` (default: torch's current stream).
+    """
+    _check_inputs(q, k, v, device_expected=True)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor shaped like q")
+    if tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor")
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        rc = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                          lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                          _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd")
+    return out, lse
+
+
+def host_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(load_library().attn_fwd_host_workspace_bytes(B, H, N, d))
+
+
+def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+                  scale: float | None = None, out: torch.Tensor | None = None,
+                  lse: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                  device=None, stream=None, synchronize: bool = True):
+    """The same operation on CPU tensors (pinned for asynchronous copies).
+
+    The library copies q, k, v to `workspace` on the device, runs the kernel
+    and copies o and lse back, all on one stream.  Returns (o, lse) as CPU
+    tensors; with synchronize=False the caller must synchronise the stream.
+    """
+    _check_inputs(q, k, v, device_expected=False)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    pin = q.is_pinned()
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=pin)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, pin_memory=pin)
+    need = host_workspace_bytes(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+    lib = load_library()
+    with torch.cuda.device(device):
+        handle = _stream_handle(stream)
+        rc = lib.attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                               lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                               workspace.data_ptr(), workspace.numel(), handle)
+        if rc != ATTN_OK:
+            raise AttnError(rc, "attn_fwd_host")
+        if synchronize:
+            if stream is None:
+                torch.cuda.current_stream(device).synchronize()
+            elif hasattr(stream, "synchronize"):
+                stream.synchronize()
+            else:
+                torch.cuda.synchronize(device)
+    return out, lse
+
+
+def device_status(reset: bool = True, stream=None) -> int:
+    """Synchronise `stream` and return (and by default clear) the device
+    status word: 0, or the first in-kernel error code recorded."""
+    return int(load_library().attn_device_status(_stream_handle(stream), int(bool(reset))))

@@ -1,0 +1,960 @@
+/*
+ * attn_fwd_sm100.cu -- fused exact-attention forward for B200 (sm_100a) and
+ * the C ABI around it.
+ *
+ * What is computed (FlashAttention teaching pages): per head,
+ *   O = softmax(scale * Q K^T [+ causal mask]) V  and  LSE_i = ln sum_j e^{s_ij}
+ * ("GPU 学习日报 Day 21", sections 3.1 and 5.3; the saved statistic of airsota
+ * "science-depth-m4-047", section 3 point (c)).  The N x N matrices S and P
+ * exist only tile by tile on chip (page 2, section 4): S in tensor memory
+ * (TMEM), P overwriting S in TMEM as bf16, never in device memory.
+ *
+ * How it maps onto sm_100a (one persistent CTA per SM, 10 warps):
+ *   warp 8      TMA producer: Q tiles once per work unit, then K_j, V_j through
+ *               a ring of shared-memory stages guarded by mbarriers.
+ *   warp 9      MMA issuer (one thread): tcgen05.mma S_t = Q_t K_j^T into TMEM
+ *               (both operands in shared memory), then O_t += P_t V_j with P_t
+ *               read from TMEM and V_j from shared memory.  It also owns the
+ *               TMEM allocation (512 columns).
+ *   warps 0-3   softmax for Q tile 0; warps 4-7 softmax for Q tile 1.  Thread
+ *               r owns row r of its tile, which is TMEM lane r, so the row max
+ *               and row sum need no shuffles.  Online recurrence of page 2,
+ *               section 5.3, in base 2 with log2(e) folded into the scale,
+ *               with lazy rescaling: the reference max only moves when a block
+ *               max exceeds it by more than TAU (so e^{s-m} <= 2^TAU), which is
+ *               exact because numerator and denominator share the reference
+ *               (page 2, section 5.2).  At the end of a unit the same warps
+ *               divide O by l, round to bf16 and store O and LSE.
+ *   A work unit is a pair of 128-row Q tiles of one head; the two tiles share
+ *   every K/V block and ping-pong on the tensor core (while one tile's softmax
+ *   runs, the other tile's GEMMs run).  Causal: blocks above the diagonal are
+ *   never loaded or computed; only the diagonal block is masked element-wise
+ *   (page 2, section 6 table).  Units are ordered longest first and dealt to
+ *   the persistent CTAs in snake order.
+ *
+ * Every wait on an mbarrier is bounded (iterations and wall time); when one
+ * runs out the CTA records ATTN_ERR_TIMEOUT in a device status word, raises an
+ * abort flag that the other warps see, waits (bounded) for its own copies and
+ * MMAs in flight, frees its TMEM and exits.
+ */
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "attn_fwd.h"
+
+#define ATTN_VERSION "0.1.0"
+
+namespace {
+
+/* ------------------------------------------------------------------------ */
+/* Tile configuration                                                        */
+/* ------------------------------------------------------------------------ */
+constexpr int BLOCK_M = 128;          // query rows per Q tile = TMEM lanes
+constexpr int BLOCK_N = 128;          // key/value rows per K/V block
+constexpr int UNIT_ROWS = 2 * BLOCK_M;  // a work unit = two Q tiles
+constexpr int NUM_THREADS = 320;
+constexpr int LOAD_WARP = 8;
+constexpr int MMA_WARP = 9;
+constexpr int TMEM_COLS = 512;
+constexpr int CHUNK_ELEMS = 64;                     // one 128-byte swizzle atom of bf16
+constexpr int CHUNK_BYTES = BLOCK_M * 128;          // 128 rows x 128 bytes
+constexpr float TAU = 8.0f;           // lazy-rescale threshold, log2 units
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s
+constexpr uint32_t WAIT_MAX_ITERS = 1u << 28;
+constexpr float LN2 = 0.6931471805599453f;
+constexpr float LOG2E = 1.4426950408889634f;
+
+template <int D>
+struct Cfg {
+    static constexpr int TILE_BYTES = BLOCK_M * D * 2;   // 128 rows x D bf16
+    static constexpr int CHUNKS = D / CHUNK_ELEMS;       // swizzle atoms along d
+    static constexpr int NSTAGE = (D == 128) ? 4 : 8;    // K/V ring slots
+    static constexpr int Q_OFF = 0;
+    static constexpr int RING_OFF = 2 * TILE_BYTES;
+    static constexpr int BAR_OFF = RING_OFF + NSTAGE * TILE_BYTES;
+    static constexpr int NUM_BARS = 2 + 2 * NSTAGE + 6 + 1;
+    static constexpr int MISC_OFF = BAR_OFF + 8 * NUM_BARS;
+    static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
+    // TMEM columns: S/P of tile t at 128*t, O of tile t at 256 + D*t
+    static constexpr uint32_t S_COL0 = 0, S_COL1 = 128;
+    static constexpr uint32_t O_COL0 = 256, O_COL1 = 256 + D;
+    static_assert(D == 64 || D == 128, "head dim");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+struct FwdParams {
+    __nv_bfloat16* o;
+    float* lse;
+    int N;          // sequence length
+    int BH;         // B * H
+    int n_pairs;    // ceil(N / 256)
+    int nkv;        // ceil(N / 128)
+    int n_units;    // BH * n_pairs
+    float scale_log2;  // scale * log2(e)
+};
+
+__device__ int g_attn_status = 0;
+
+/* ------------------------------------------------------------------------ */
+/* PTX wrappers                                                              */
+/* ------------------------------------------------------------------------ */
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void record_error(int code) { atomicCAS(&g_attn_status, 0, code); }
+
+/* Bounded wait for the phase of parity `parity` of an mbarrier.  Returns false
+ * when another warp raised the abort flag, or after the limit (then it records
+ * the timeout and raises the flag itself). */
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag) {
+    if (mbar_try(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 0; it < WAIT_MAX_ITERS; ++it) {
+        if (mbar_try(bar, parity)) return true;
+        if ((it & 63u) == 63u) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > WAIT_LIMIT_NS) break;
+        }
+    }
+    record_error(ATTN_ERR_TIMEOUT);
+    *abort_flag = 1u;
+    return false;
+}
+
+/* Bounded wait that ignores the abort flag: used on the abort path to let the
+ * CTA's own copies and MMAs in flight land before it exits. */
+__device__ __noinline__ void mbar_drain_wait(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 0; it < WAIT_MAX_ITERS; ++it) {
+        if (mbar_try(bar, parity)) return;
+        if ((it & 63u) == 63u && globaltimer() - t0 > WAIT_LIMIT_NS) return;
+    }
+}
+
+__device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint32_t dst, uint32_t bar,
+                                            int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+/* Shared-memory matrix descriptor for tcgen05.mma, 128-byte swizzle.
+ * Bits: [0,14) start >> 4, [16,30) leading byte offset >> 4, [32,46) stride
+ * byte offset >> 4, [46,48) version (1 on sm_100), [61,64) layout (2 = 128B swizzle). */
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
+/* Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, dense.
+ * Bits: [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format,
+ * 15 A major (0 = K), 16 B major (1 = MN), [17,23) N >> 3, [24,29) M >> 4. */
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+/* Two fp32 -> one bf16x2 word, round to nearest even; `lo` in bits 0-15. */
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+/* tcgen05.ld of 128 consecutive 32-bit columns of this thread's TMEM lane, with
+ * the wait in the same asm statement so no use of v[] can be scheduled early. */
+__device__ __forceinline__ void tmem_ld128_wait(uint32_t taddr, uint32_t* v) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x128.b32 {"
+        "%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+        "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+        "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, "
+        "%64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, "
+        "%80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, "
+        "%96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, "
+        "%112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127"
+        "}, [%128];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31]),
+          "=r"(v[32]), "=r"(v[33]), "=r"(v[34]), "=r"(v[35]), "=r"(v[36]), "=r"(v[37]), "=r"(v[38]), "=r"(v[39]),
+          "=r"(v[40]), "=r"(v[41]), "=r"(v[42]), "=r"(v[43]), "=r"(v[44]), "=r"(v[45]), "=r"(v[46]), "=r"(v[47]),
+          "=r"(v[48]), "=r"(v[49]), "=r"(v[50]), "=r"(v[51]), "=r"(v[52]), "=r"(v[53]), "=r"(v[54]), "=r"(v[55]),
+          "=r"(v[56]), "=r"(v[57]), "=r"(v[58]), "=r"(v[59]), "=r"(v[60]), "=r"(v[61]), "=r"(v[62]), "=r"(v[63]),
+          "=r"(v[64]), "=r"(v[65]), "=r"(v[66]), "=r"(v[67]), "=r"(v[68]), "=r"(v[69]), "=r"(v[70]), "=r"(v[71]),
+          "=r"(v[72]), "=r"(v[73]), "=r"(v[74]), "=r"(v[75]), "=r"(v[76]), "=r"(v[77]), "=r"(v[78]), "=r"(v[79]),
+          "=r"(v[80]), "=r"(v[81]), "=r"(v[82]), "=r"(v[83]), "=r"(v[84]), "=r"(v[85]), "=r"(v[86]), "=r"(v[87]),
+          "=r"(v[88]), "=r"(v[89]), "=r"(v[90]), "=r"(v[91]), "=r"(v[92]), "=r"(v[93]), "=r"(v[94]), "=r"(v[95]),
+          "=r"(v[96]), "=r"(v[97]), "=r"(v[98]), "=r"(v[99]), "=r"(v[100]), "=r"(v[101]), "=r"(v[102]), "=r"(v[103]),
+          "=r"(v[104]), "=r"(v[105]), "=r"(v[106]), "=r"(v[107]), "=r"(v[108]), "=r"(v[109]), "=r"(v[110]), "=r"(v[111]),
+          "=r"(v[112]), "=r"(v[113]), "=r"(v[114]), "=r"(v[115]), "=r"(v[116]), "=r"(v[117]), "=r"(v[118]), "=r"(v[119]),
+          "=r"(v[120]), "=r"(v[121]), "=r"(v[122]), "=r"(v[123]), "=r"(v[124]), "=r"(v[125]), "=r"(v[126]), "=r"(v[127])
+        : "r"(taddr)
+        : "memory");
+}
+
+/* tcgen05.ld of 32 consecutive 32-bit columns of this thread's TMEM lane, with
+ * the wait in the same asm statement so no use of v[] can be scheduled early. */
+__device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t* v) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
+        "%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31"
+        "}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+/* tcgen05.st of 32 consecutive 32-bit columns into this thread's TMEM lane. */
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {"
+        "%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32"
+        "};"
+        :
+        : "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+          "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+          "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+/* ------------------------------------------------------------------------ */
+/* Work units and the static schedule                                        */
+/* ------------------------------------------------------------------------ */
+struct Unit {
+    int bh;     // flat head index b*H + h
+    int pair;   // Q rows [256*pair, 256*pair + 256)
+    int n[2];   // K/V blocks Q tile t needs (0 when the tile lies past N)
+};
+
+/* Causal units are ordered by decreasing work (pair index descending, heads
+ * minor); non-causal units head-major so concurrent CTAs share K/V in L2. */
+template <bool CAUSAL>
+__device__ __forceinline__ Unit unit_at(int idx, const FwdParams& p) {
+    Unit u;
+    if (CAUSAL) {
+        u.pair = p.n_pairs - 1 - idx / p.BH;
+        u.bh = idx % p.BH;
+    } else {
+        u.bh = idx / p.n_pairs;
+        u.pair = idx % p.n_pairs;
+    }
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int r0 = u.pair * UNIT_ROWS + t * BLOCK_M;
+        if (r0 >= p.N) {
+            u.n[t] = 0;
+        } else if (CAUSAL) {
+            const int last = r0 / BLOCK_N;          // the diagonal block of this tile
+            u.n[t] = last + 1 < p.nkv ? last + 1 : p.nkv;
+        } else {
+            u.n[t] = p.nkv;
+        }
+    }
+    return u;
+}
+
+/* Snake deal: round r gives CTA c the unit r*G + c (r even) or r*G + G-1-c
+ * (r odd), so each CTA's list mixes long and short units. */
+__device__ __forceinline__ int unit_index(int round) {
+    const int G = gridDim.x, c = blockIdx.x;
+    return round * G + ((round & 1) ? (G - 1 - c) : c);
+}
+
+/* ------------------------------------------------------------------------ */
+/* The kernel                                                                */
+/* ------------------------------------------------------------------------ */
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+    using C = Cfg<D>;
+    constexpr int NSTAGE = C::NSTAGE;
+    constexpr uint32_t TILE = C::TILE_BYTES;
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;   // 128B swizzle needs 1024B-aligned tiles
+    uint8_t* const base_ptr = smem_raw + (base - raw);
+
+    const uint32_t sQ[2] = {base + C::Q_OFF, base + C::Q_OFF + TILE};
+    const uint32_t sRing = base + C::RING_OFF;
+    const uint32_t bars = base + C::BAR_OFF;
+    const uint32_t bar_q_full = bars;
+    const uint32_t bar_q_empty = bars + 8;
+    auto bar_kv_full = [&](int s) { return bars + 16 + 8u * s; };
+    auto bar_kv_empty = [&](int s) { return bars + 16 + 8u * (NSTAGE + s); };
+    const uint32_t bar_s_full0 = bars + 16 + 16 * NSTAGE;      // [2]
+    const uint32_t bar_p_ready0 = bar_s_full0 + 16;            // [2]
+    const uint32_t bar_o_full0 = bar_p_ready0 + 16;            // [2]
+    const uint32_t bar_drain = bar_o_full0 + 16;
+    uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::MISC_OFF);
+    volatile uint32_t* const abort_flag = reinterpret_cast<volatile uint32_t*>(base_ptr + C::MISC_OFF + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q_full, 1);
+        mbar_init(bar_q_empty, 1);
+        for (int s = 0; s < NSTAGE; ++s) {
+            mbar_init(bar_kv_full(s), 1);
+            mbar_init(bar_kv_empty(s), 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bar_s_full0 + 8 * t, 1);
+            mbar_init(bar_p_ready0 + 8 * t, BLOCK_M);   // every softmax thread of the tile
+            mbar_init(bar_o_full0 + 8 * t, 1);
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == LOAD_WARP && lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+    }
+    if (warp == MMA_WARP) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == LOAD_WARP) {
+        /* ---------------- TMA producer ---------------- */
+        if (lane == 0) {
+            uint32_t it = 0;          // K/V ring position (K_j and V_j each take one)
+            int local = 0;            // units this CTA has started
+            bool aborted = false;
+            for (int r = 0;; ++r) {
+                const int idx = unit_index(r);
+                if (idx >= p.n_units) break;
+                const Unit u = unit_at<CAUSAL>(idx, p);
+                if (local > 0 && !mbar_wait(bar_q_empty, (local - 1) & 1, abort_flag)) {
+                    aborted = true;
+                    break;
+                }
+                mbar_arrive_expect_tx(bar_q_full, 2 * TILE);
+                for (int t = 0; t < 2; ++t)
+                    for (int c = 0; c < C::CHUNKS; ++c)
+                        tma_load_3d(&tm_q, sQ[t] + c * CHUNK_BYTES, bar_q_full, c * CHUNK_ELEMS,
+                                    u.pair * UNIT_ROWS + t * BLOCK_M, u.bh);
+                const int nmax = u.n[0] > u.n[1] ? u.n[0] : u.n[1];
+                for (int j = 0; j < nmax && !aborted; ++j) {
+                    for (int kv = 0; kv < 2; ++kv) {
+                        const int s = it % NSTAGE;
+                        const uint32_t use = it / NSTAGE;
+                        if (!mbar_wait(bar_kv_empty(s), (use & 1u) ^ 1u, abort_flag)) {
+                            aborted = true;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(bar_kv_full(s), TILE);
+                        const CUtensorMap* m = kv ? &tm_v : &tm_k;
+                        for (int c = 0; c < C::CHUNKS; ++c)
+                            tma_load_3d(m, sRing + s * TILE + c * CHUNK_BYTES, bar_kv_full(s),
+                                        c * CHUNK_ELEMS, j * BLOCK_N, u.bh);
+                        ++it;
+                    }
+                }
+                ++local;
+                if (aborted) break;
+            }
+            if (aborted) {
+                /* let this CTA's copies in flight land before the CTA exits */
+                if (local > 0) mbar_drain_wait(bar_q_full, (local - 1) & 1);
+                const uint32_t n_back = it < (uint32_t)NSTAGE ? it : (uint32_t)NSTAGE;
+                for (uint32_t b = 1; b <= n_back; ++b) {
+                    const uint32_t i = it - b;
+                    mbar_drain_wait(bar_kv_full(i % NSTAGE), (i / NSTAGE) & 1u);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == MMA_WARP) {
+        /* ---------------- MMA issuer ---------------- */
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16(BLOCK_M, BLOCK_N, false);
+            constexpr uint32_t IDESC_PV = idesc_bf16(BLOCK_M, D, true);
+            const uint32_t s_col[2] = {C::S_COL0, C::S_COL1};
+            const uint32_t o_col[2] = {C::O_COL0, C::O_COL1};
+            uint32_t it = 0;
+            uint32_t pr[2] = {0, 0};   // p_ready phases consumed per tile
+            int local = 0;
+
+            // S_t = Q_t K^T for the K block in ring slot `slot`
+            auto issue_s = [&](int t, int slot) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32;
+                    const uint64_t a = sdesc_sw128(sQ[t] + koff, 16, 1024);
+                    const uint64_t b = sdesc_sw128(sRing + slot * TILE + koff, 16, 1024);
+                    mma_ss(tmem + s_col[t], a, b, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+            };
+            // O_t (+)= P_t V for the V block in ring slot `slot`; P_t is bf16 in TMEM
+            auto issue_pv = [&](int t, int slot, bool acc) {
+#pragma unroll
+                for (int kk = 0; kk < BLOCK_N / 16; ++kk) {
+                    const uint64_t b = sdesc_sw128(sRing + slot * TILE + kk * 16 * 128,
+                                                   CHUNK_BYTES, 1024);
+                    mma_ts(tmem + o_col[t], tmem + s_col[t] + kk * 8, b, IDESC_PV,
+                           (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+
+            bool aborted = false;
+            for (int r = 0; !aborted; ++r) {
+                const int idx = unit_index(r);
+                if (idx >= p.n_units) break;
+                const Unit u = unit_at<CAUSAL>(idx, p);
+                const int n0 = u.n[0], n1 = u.n[1];
+                const int nmax = n0 > n1 ? n0 : n1;
+                if (!mbar_wait(bar_q_full, local & 1, abort_flag)) { aborted = true; break; }
+                tc_fence_after();
+                // K_0
+                {
+                    const int ks = it % NSTAGE;
+                    if (!mbar_wait(bar_kv_full(ks), (it / NSTAGE) & 1u, abort_flag)) { aborted = true; break; }
+                    tc_fence_after();
+                    if (n0 > 0) { issue_s(0, ks); mma_commit(bar_s_full0); }
+                    if (n1 > 0) { issue_s(1, ks); mma_commit(bar_s_full0 + 8); }
+                    if (nmax == 1) mma_commit(bar_q_empty);
+                    mma_commit(bar_kv_empty(ks));
+                    ++it;
+                }
+                for (int j = 0; j < nmax; ++j) {
+                    const int vs = it % NSTAGE;
+                    if (!mbar_wait(bar_kv_full(vs), (it / NSTAGE) & 1u, abort_flag)) { aborted = true; break; }
+                    tc_fence_after();
+                    ++it;
+                    const bool has_next = j + 1 < nmax;
+                    const int ks = it % NSTAGE;
+                    bool k_ready = false;
+                    if (j < n0) {
+                        if (!mbar_wait(bar_p_ready0, pr[0] & 1u, abort_flag)) { aborted = true; break; }
+                        ++pr[0];
+                        tc_fence_after();
+                        issue_pv(0, vs, j > 0);
+                        if (j == n0 - 1) mma_commit(bar_o_full0);
+                    }
+                    if (j + 1 < n0) {
+                        if (!mbar_wait(bar_kv_full(ks), (it / NSTAGE) & 1u, abort_flag)) { aborted = true; break; }
+                        tc_fence_after();
+                        k_ready = true;
+                        issue_s(0, ks);
+                        mma_commit(bar_s_full0);
+                    }
+                    if (j < n1) {
+                        if (!mbar_wait(bar_p_ready0 + 8, pr[1] & 1u, abort_flag)) { aborted = true; break; }
+                        ++pr[1];
+                        tc_fence_after();
+                        issue_pv(1, vs, j > 0);
+                        if (j == n1 - 1) mma_commit(bar_o_full0 + 8);
+                    }
+                    mma_commit(bar_kv_empty(vs));
+                    if (has_next) {
+                        if (!k_ready) {
+                            if (!mbar_wait(bar_kv_full(ks), (it / NSTAGE) & 1u, abort_flag)) { aborted = true; break; }
+                            tc_fence_after();
+                        }
+                        if (j + 1 < n1) { issue_s(1, ks); mma_commit(bar_s_full0 + 8); }
+                        if (j + 1 == nmax - 1) mma_commit(bar_q_empty);
+                        mma_commit(bar_kv_empty(ks));
+                        ++it;
+                    }
+                }
+                ++local;
+            }
+            /* all MMAs this thread issued have completed once this phase lands */
+            mma_commit(bar_drain);
+            mbar_drain_wait(bar_drain, 0);
+        }
+        __syncwarp();
+    } else {
+        /* ---------------- softmax + epilogue, warps 0-7 ---------------- */
+        const int t = warp >> 2;                 // Q tile of this warpgroup
+        const int quarter = warp & 3;            // TMEM lanes [32*quarter, 32*quarter + 32)
+        const int row_in_tile = quarter * 32 + lane;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const uint32_t s_addr = lane_base + (t ? C::S_COL1 : C::S_COL0);
+        const uint32_t o_addr = lane_base + (t ? C::O_COL1 : C::O_COL0);
+        const uint32_t bar_s = bar_s_full0 + 8 * t;
+        const uint32_t bar_p = bar_p_ready0 + 8 * t;
+        const uint32_t bar_o = bar_o_full0 + 8 * t;
+        const float c = p.scale_log2;
+        uint32_t sph = 0, oph = 0;
+        const int tail = p.N & (BLOCK_N - 1);   // valid keys in the last block (0 = full)
+
+        for (int r = 0;; ++r) {
+            const int idx = unit_index(r);
+            if (idx >= p.n_units) break;
+            const Unit u = unit_at<CAUSAL>(idx, p);
+            const int n = u.n[t];
+            if (n == 0) continue;
+            const int row = u.pair * UNIT_ROWS + t * BLOCK_M + row_in_tile;
+            float m_ref = -INFINITY;   // reference max, log2 units of scale*q.k
+            float l = 0.0f;            // running sum of 2^(c*s - m_ref)
+            bool ok = true;
+            for (int j = 0; j < n; ++j) {
+                ok = mbar_wait(bar_s, sph & 1u, abort_flag);
+                ++sph;
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t sraw[BLOCK_N];
+                tmem_ld128_wait(s_addr, sraw);
+                float* s = reinterpret_cast<float*>(sraw);
+                if (CAUSAL && j == n - 1) {
+                    // diagonal block: key column cc masked when cc > row_in_tile
+#pragma unroll
+                    for (int cc = 0; cc < BLOCK_N; ++cc)
+                        if (cc > row_in_tile) s[cc] = -INFINITY;
+                } else if (!CAUSAL && tail != 0 && j == n - 1) {
+#pragma unroll
+                    for (int cc = 0; cc < BLOCK_N; ++cc)
+                        if (cc >= tail) s[cc] = -INFINITY;
+                }
+                float mx = s[0];
+#pragma unroll
+                for (int cc = 1; cc < BLOCK_N; ++cc) mx = fmaxf(mx, s[cc]);
+                const float mb = mx * c;               // block max, log2 units
+                const bool need = mb > m_ref + TAU;
+                float alpha = 1.0f;
+                if (need) {
+                    alpha = ex2(m_ref - mb);           // 0 on the first block
+                    l *= alpha;
+                    m_ref = mb;
+                }
+                const float neg_m = (m_ref == -INFINITY) ? 0.0f : -m_ref;
+                uint32_t pk[BLOCK_N / 2];
+                float sum0 = 0.0f, sum1 = 0.0f;
+#pragma unroll
+                for (int cc = 0; cc < BLOCK_N / 2; ++cc) {
+                    const float p0 = ex2(fmaf(s[2 * cc], c, neg_m));
+                    const float p1 = ex2(fmaf(s[2 * cc + 1], c, neg_m));
+                    sum0 += p0;
+                    sum1 += p1;
+                    pk[cc] = pack_bf16(p0, p1);
+                }
+                l += sum0 + sum1;
+                tmem_st32(s_addr, pk);
+                tmem_st32(s_addr + 32, pk + 32);
+                if (j > 0 && __any_sync(0xffffffffu, need)) {
+                    // rescale this row of O_acc in TMEM (PV of block j-1 has
+                    // completed: the commit that released S_j covers it)
+#pragma unroll
+                    for (int ch = 0; ch < D / 32; ++ch) {
+                        uint32_t ov[32];
+                        tmem_ld32_wait(o_addr + ch * 32, ov);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                        tmem_st32(o_addr + ch * 32, ov);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar_p);
+            }
+            if (!ok) break;
+            ok = mbar_wait(bar_o, oph & 1u, abort_flag);
+            ++oph;
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
+            const bool live = row < p.N;
+            __nv_bfloat16* orow = p.o + (static_cast<size_t>(u.bh) * p.N + (live ? row : 0)) * D;
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t ov[32];
+                tmem_ld32_wait(o_addr + ch * 32, ov);
+                uint32_t w[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    w[e] = pack_bf16(__uint_as_float(ov[2 * e]) * inv_l,
+                                     __uint_as_float(ov[2 * e + 1]) * inv_l);
+                if (live) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                }
+            }
+            if (live) p.lse[static_cast<size_t>(u.bh) * p.N + row] = (m_ref + log2f(l)) * LN2;
+            tc_fence_before();
+        }
+    }
+
+    /* ---------------- teardown ---------------- */
+    tc_fence_before();
+    __syncthreads();
+    if (warp == MMA_WARP) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+}  // namespace
+/* ------------------------------------------------------------------------ */
+/* Host side: validation, tensor maps, launch                                */
+/* ------------------------------------------------------------------------ */
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+constexpr int MAX_DEVICES = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    int status = ATTN_OK;   // ATTN_ERR_DEVICE when the device is not CC 10.0
+    int num_sms = 0;
+    bool smem_set[4] = {false, false, false, false};
+};
+
+std::mutex g_mutex;
+DeviceInfo g_dev[MAX_DEVICES];
+EncodeTiledFn g_encode = nullptr;
+
+int get_encode(EncodeTiledFn* fn) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_encode) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult qres;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) !=
+                cudaSuccess ||
+            qres != cudaDriverEntryPointSuccess || !ptr) {
+            cudaGetLastError();
+            return ATTN_ERR_CUDA;
+        }
+        g_encode = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    *fn = g_encode;
+    return ATTN_OK;
+}
+
+int device_info(int* dev_out, DeviceInfo** info_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return ATTN_ERR_CUDA; }
+    if (dev < 0 || dev >= MAX_DEVICES) return ATTN_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo& di = g_dev[dev];
+    if (!di.ready) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return ATTN_ERR_CUDA;
+        }
+        di.status = (major == 10 && minor == 0) ? ATTN_OK : ATTN_ERR_DEVICE;
+        di.num_sms = sms;
+        di.ready = true;
+    }
+    *dev_out = dev;
+    *info_out = &di;
+    return di.status;
+}
+
+/* 3-D view [B*H][N][d] of a bf16 tensor, box = 64 columns x 128 rows x 1 head,
+ * 128-byte swizzle; rows past N read as zeros. */
+int encode_map(EncodeTiledFn fn, CUtensorMap* map, const void* ptr, int64_t BH, int64_t N,
+               int64_t d) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                          static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(N * d * 2)};
+    cuuint32_t box[3] = {CHUNK_ELEMS, BLOCK_M, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+/* Argument checks shared by the device and host entry points (no CUDA calls). */
+int validate_shape(int64_t B, int64_t H, int64_t N, int64_t d, float scale, bool* empty) {
+    if (B < 0 || H < 0 || N < 0) return ATTN_ERR_SHAPE;
+    if (d != 64 && d != 128) return ATTN_ERR_HEADDIM;
+    if (!(scale > 0.0f) || !isfinite(scale)) return ATTN_ERR_SCALE;
+    *empty = (B == 0 || H == 0 || N == 0);
+    if (*empty) return ATTN_OK;
+    if (N > INT32_MAX - 2 * UNIT_ROWS) return ATTN_ERR_SHAPE;
+    if (H > INT32_MAX / B) return ATTN_ERR_SHAPE;
+    const int64_t BH = B * H;
+    const int64_t n_pairs = (N + UNIT_ROWS - 1) / UNIT_ROWS;
+    if (BH > INT32_MAX / n_pairs) return ATTN_ERR_SHAPE;   // unit index fits int32
+    return ATTN_OK;
+}
+
+template <int D, bool CAUSAL>
+int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+           const FwdParams& prm, DeviceInfo* di, cudaStream_t stream) {
+    auto kern = attn_fwd_sm100_kernel<D, CAUSAL>;
+    constexpr int SMEM = Cfg<D>::SMEM_BYTES;
+    const int key = (D == 128 ? 2 : 0) + (CAUSAL ? 1 : 0);
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!di->smem_set[key]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
+                cudaSuccess) {
+                cudaGetLastError();
+                return ATTN_ERR_LAUNCH;
+            }
+            di->smem_set[key] = true;
+        }
+    }
+    const int grid = prm.n_units < di->num_sms ? prm.n_units : di->num_sms;
+    kern<<<grid, NUM_THREADS, SMEM, stream>>>(mq, mk, mv, prm);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+    return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+             int64_t H, int64_t N, int64_t d, int causal, float scale, void* stream) {
+    bool empty = false;
+    int st = validate_shape(B, H, N, d, scale, &empty);
+    if (st != ATTN_OK || empty) return st;
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
+    const void* ptrs[5] = {q, k, v, o, lse};
+    for (const void* ptr : ptrs)
+        if (reinterpret_cast<uintptr_t>(ptr) & 15u) return ATTN_ERR_ALIGN;
+    const size_t tbytes = static_cast<size_t>(B * H * N * d) * 2;
+    const size_t lbytes = static_cast<size_t>(B * H * N) * 4;
+    if (ranges_overlap(o, tbytes, q, tbytes) || ranges_overlap(o, tbytes, k, tbytes) ||
+        ranges_overlap(o, tbytes, v, tbytes) || ranges_overlap(lse, lbytes, q, tbytes) ||
+        ranges_overlap(lse, lbytes, k, tbytes) || ranges_overlap(lse, lbytes, v, tbytes) ||
+        ranges_overlap(lse, lbytes, o, tbytes))
+        return ATTN_ERR_OVERLAP;
+
+    int dev = 0;
+    DeviceInfo* di = nullptr;
+    if ((st = device_info(&dev, &di)) != ATTN_OK) return st;
+    EncodeTiledFn enc = nullptr;
+    if ((st = get_encode(&enc)) != ATTN_OK) return st;
+    const int64_t BH = B * H;
+    CUtensorMap mq, mk, mv;
+    if ((st = encode_map(enc, &mq, q, BH, N, d)) != ATTN_OK) return st;
+    if ((st = encode_map(enc, &mk, k, BH, N, d)) != ATTN_OK) return st;
+    if ((st = encode_map(enc, &mv, v, BH, N, d)) != ATTN_OK) return st;
+
+    FwdParams prm;
+    prm.o = static_cast<__nv_bfloat16*>(o);
+    prm.lse = lse;
+    prm.N = static_cast<int>(N);
+    prm.BH = static_cast<int>(BH);
+    prm.n_pairs = static_cast<int>((N + UNIT_ROWS - 1) / UNIT_ROWS);
+    prm.nkv = static_cast<int>((N + BLOCK_N - 1) / BLOCK_N);
+    prm.n_units = prm.BH * prm.n_pairs;
+    prm.scale_log2 = scale * LOG2E;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (d == 64)
+        return causal ? launch<64, true>(mq, mk, mv, prm, di, s) : launch<64, false>(mq, mk, mv, prm, di, s);
+    return causal ? launch<128, true>(mq, mk, mv, prm, di, s) : launch<128, false>(mq, mk, mv, prm, di, s);
+}
+
+static size_t align256(size_t x) { return (x + 255u) & ~static_cast<size_t>(255u); }
+
+size_t attn_fwd_host_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {
+    bool empty = false;
+    if (validate_shape(B, H, N, d, 1.0f, &empty) != ATTN_OK) return 0;
+    const size_t tbytes = static_cast<size_t>(B * H * N * d) * 2;
+    const size_t lbytes = static_cast<size_t>(B * H * N) * 4;
+    return 4 * align256(tbytes) + align256(lbytes);
+}
+
+int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+                  int64_t H, int64_t N, int64_t d, int causal, float scale, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+    bool empty = false;
+    int st = validate_shape(B, H, N, d, scale, &empty);
+    if (st != ATTN_OK || empty) return st;
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+        workspace_bytes < attn_fwd_host_workspace_bytes(B, H, N, d))
+        return ATTN_ERR_WORKSPACE;
+    const size_t tbytes = static_cast<size_t>(B * H * N * d) * 2;
+    const size_t lbytes = static_cast<size_t>(B * H * N) * 4;
+    char* ws = static_cast<char*>(workspace);
+    void* dq = ws;
+    void* dk = ws + align256(tbytes);
+    void* dv = ws + 2 * align256(tbytes);
+    void* dout = ws + 3 * align256(tbytes);
+    float* dl = reinterpret_cast<float*>(ws + 4 * align256(tbytes));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(dq, q, tbytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dk, k, tbytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dv, v, tbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    if ((st = attn_fwd(dq, dk, dv, dout, dl, B, H, N, d, causal, scale, stream)) != ATTN_OK)
+        return st;
+    if (cudaMemcpyAsync(o, dout, tbytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemcpyAsync(lse, dl, lbytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
+}
+
+int attn_device_status(void* stream, int reset) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_attn_status, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    if (reset) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_attn_status, &zero, sizeof(int)) != cudaSuccess) {
+            cudaGetLastError();
+            return ATTN_ERR_CUDA;
+        }
+    }
+    return v;
+}
+
+const char* attn_status_str(int status) {
+    switch (status) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_NULL: return "a required pointer is NULL";
+        case ATTN_ERR_ALIGN: return "a device pointer is not 16-byte aligned";
+        case ATTN_ERR_HEADDIM: return "head dimension must be 64 or 128";
+        case ATTN_ERR_SHAPE: return "B, H or N out of range";
+        case ATTN_ERR_SCALE: return "scale must be finite and > 0";
+        case ATTN_ERR_DEVICE: return "current device is not an sm_100 (compute capability 10.0) GPU";
+        case ATTN_ERR_LAUNCH: return "kernel launch failed";
+        case ATTN_ERR_TIMEOUT: return "a bounded wait inside the kernel ran out";
+        case ATTN_ERR_CUDA: return "CUDA runtime or driver error";
+        case ATTN_ERR_OVERLAP: return "an output buffer overlaps an input or the other output";
+        case ATTN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        default: return "unknown status";
+    }
+}
+
+const char* attn_version(void) { return ATTN_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,113 @@
+/*
+ * attn_fwd.h -- C ABI of the B200 (sm_100a) exact-attention forward library.
+ *
+ * The operation (FlashAttention teaching pages):
+ *   "GPU 学习日报 Day 21", section 3.1, states the problem per head:
+ *       S = Q K^T / sqrt(d),  P = softmax(S),  O = P V.
+ *   Here the score scale is an argument, and an optional causal mask drops key
+ *   j from query row i whenever j > i (the same page, section 6 table, row on
+ *   causal-mask waste).  The forward pass also returns, per query row, the
+ *   statistic the backward pass recomputes from (airsota "science-depth-m4-047",
+ *   section 3, point (c)), read as the natural-log log-sum-exp
+ *       LSE_i = ln( sum_{j allowed} exp(scale * q_i . k_j) ).
+ *   The result is computed as in sections 4-5 of page 2: one fused kernel that
+ *   tiles Q, K and V through on-chip memory with the online-softmax recurrence,
+ *   so the N x N score and probability matrices never reach device memory.
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are dense and row-major: q, k, v, o are bf16 [B, H, N, d] with d
+ *     contiguous; lse is fp32 [B, H, N].  Q, K and V share one sequence length
+ *     N (self-attention; the causal mask is aligned at the top-left corner).
+ *   - d must be 64 or 128.  B, H, N >= 1; B*H < 2^31; N < 2^31.  A call with
+ *     B*H*N == 0 is not an error: it returns ATTN_OK and launches nothing.
+ *   - scale must be finite and > 0 (1/sqrt(d) is the usual choice).
+ *   - Device pointers must be 16-byte aligned (the tensor-memory-accelerator
+ *     copies require it).  o and lse must not overlap q, k, v or each other.
+ *   - The caller owns every buffer.  These calls allocate no device memory.
+ *   - stream is a cudaStream_t passed as void*; NULL means the legacy default
+ *     stream.  A device call is asynchronous on that stream; a non-zero return
+ *     means nothing was launched (or, for attn_fwd_host, that the sequence of
+ *     enqueued operations stopped at the failing step).
+ *   - Error behaviour: argument errors are detected on the host before any
+ *     CUDA call and returned as negative attn_status_t codes.  A device-side
+ *     fault (a bounded wait that ran out) is recorded in a per-device status
+ *     word that attn_device_status() reads and clears.
+ */
+#ifndef ATTN_FWD_H
+#define ATTN_FWD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_NULL = -1,      /* a required pointer is NULL                         */
+    ATTN_ERR_ALIGN = -2,     /* a device pointer is not 16-byte aligned            */
+    ATTN_ERR_HEADDIM = -3,   /* d is not 64 or 128                                 */
+    ATTN_ERR_SHAPE = -4,     /* B, H or N out of range                             */
+    ATTN_ERR_SCALE = -5,     /* scale not finite or not > 0                        */
+    ATTN_ERR_DEVICE = -6,    /* the current device is not compute capability 10.0  */
+    ATTN_ERR_LAUNCH = -7,    /* the kernel launch (or a copy) was refused by CUDA  */
+    ATTN_ERR_TIMEOUT = -8,   /* a bounded wait inside the kernel ran out           */
+    ATTN_ERR_CUDA = -9,      /* another CUDA runtime/driver error                  */
+    ATTN_ERR_OVERLAP = -10,  /* an output buffer overlaps an input or the other one */
+    ATTN_ERR_WORKSPACE = -11 /* workspace missing or too small                     */
+} attn_status_t;
+
+/*
+ * attn_fwd -- fused exact attention forward on device buffers.
+ *   q, k, v : device, bf16 [B, H, N, d], read only.
+ *   o       : device, bf16 [B, H, N, d], written: O = softmax(scale*QK^T [+mask]) V,
+ *             each element rounded once from fp32 to bf16 (round to nearest even).
+ *   lse     : device, fp32 [B, H, N], written: LSE_i as defined above.
+ *   causal  : 0 = every key attends; non-zero = key j is masked for row i when j > i.
+ *   scale   : multiplies q_i . k_j before the softmax.
+ * Returns ATTN_OK once the kernel is enqueued on `stream`, else an error code.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
+             void* stream);
+
+/*
+ * attn_fwd_host_workspace_bytes -- device workspace attn_fwd_host needs for a
+ * shape: room for q, k, v, o (bf16) and lse (fp32), each 256-byte aligned.
+ * Returns 0 for invalid shapes.
+ */
+size_t attn_fwd_host_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
+
+/*
+ * attn_fwd_host -- the same operation on HOST buffers.  Enqueues on `stream`:
+ * three host-to-device copies of q, k, v into `workspace` (device memory of at
+ * least attn_fwd_host_workspace_bytes), the attn_fwd kernel, and two
+ * device-to-host copies into o and lse.  Host buffers should be page-locked
+ * for the copies to be asynchronous.  The caller synchronises the stream
+ * before reading o and lse.  Same shapes, layouts and error codes as attn_fwd;
+ * the host pointers need no alignment.
+ */
+int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                  int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * attn_device_status -- read the current device's kernel status word after
+ * synchronising `stream`: ATTN_OK, or the first device-side error recorded
+ * since the last reset (ATTN_ERR_TIMEOUT).  When reset != 0 the word is
+ * cleared afterwards.  Returns ATTN_ERR_CUDA if the word cannot be read.
+ */
+int attn_device_status(void* stream, int reset);
+
+/* attn_status_str -- a static, human-readable string for a status code. */
+const char* attn_status_str(int status);
+
+/* attn_version -- library version string. */
+const char* attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_FWD_H */

@@ -1,0 +1,432 @@
+#!/usr/bin/env python
+"""Throughput of the fused attention forward on B200.
+
+One step = one call of the fused forward (the whole hot path) over one batch of
+synthetic input of the headline workload: B=4, H=16, N=8192, d=128, causal,
+scale 1/sqrt(d), bf16 inputs drawn from N(0,1) (seed 2).  The metric is forward
+TFLOP/s with FLOPs = 4*B*H*N^2*d / 2 (causal), inputs resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...      # the fp64 CPU oracle, timed
+
+With N > 1 (launched by torch.distributed.run) every rank runs its own batch
+(seed + rank): the work shards by independent problems, there is no data-path
+collective, and scaling is weak.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from exact_attention_127_b200 import inputs as _inputs  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s and % of B200 dense BF16 peak (causal N=8192 d=128)"
+UNIT = "TFLOP/s"
+DATASHEET_BF16_TFLOPS = 2250.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_NAME = "attn_fwd_sm100_kernel"
+SRC = os.path.join(ROOT, "exact_attention_127_b200", "csrc", "attn_fwd_sm100.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------------------
+# Host-side helpers (unit-tested on CPU)
+# ---------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, local, world
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own independent batch of the same shape."""
+    return int(seed) + 1000 * int(rank)
+
+
+def aggregate_value(flops_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job TFLOP/s: all ranks' useful FLOPs over the slowest rank's time."""
+    return flops_per_rank * world / (ms_max * 1e-3) / 1e12
+
+
+def reduce_max(values, device):
+    """Element-wise max over ranks of a few timings (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(x) for x in values]
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK), "fallback"
+
+
+def source_digest() -> str:
+    with open(SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def load_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu capture, or None when the
+    capture is missing, for another workload, or taken on older kernel source."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("kernel_source_sha256") != source_digest():
+        return None
+    per = rec.get("per_launch_dram_bytes", {})
+    val = per.get(workload)
+    return float(val) if val is not None else None
+
+
+REASON_BITS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+    0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+    0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+    0x100: "display_clock_setting",
+}
+
+
+def decode_reasons(mask: int):
+    return [name for bit, name in sorted(REASON_BITS.items()) if mask & bit]
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._thread = None
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception as e:  # noqa: BLE001
+            self.error = repr(e)
+
+    def _sample(self):
+        nv = self._nv
+        sm = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+        try:
+            reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        except AttributeError:
+            reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+        self.samples.append((time.time(), sm, int(reasons)))
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:  # noqa: BLE001
+                pass
+            self._stop.wait(self._period)
+
+    def start(self):
+        if self._ok:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread:
+            self._stop.set()
+            self._thread.join()
+            try:
+                self._sample()
+            except Exception:  # noqa: BLE001
+                pass
+
+    def summary(self):
+        if not self._ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0, "note": getattr(self, "error", "no samples")}
+        mhz = [s[1] for s in self.samples]
+        mask = 0
+        for s in self.samples:
+            mask |= s[2]
+        reasons = [r for r in decode_reasons(mask) if r != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(mhz), "reasons": reasons, "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle as it stands, on a bounded sample
+# ---------------------------------------------------------------------------
+def oracle_sample_flops(w, rows, n_heads):
+    """Useful FLOPs of the sampled rows: 4*d per allowed key per row."""
+    keys = sum((int(r) + 1) if w.causal else w.N for r in rows)
+    return 4.0 * w.d * keys * n_heads
+
+
+def time_oracle(w, q, k, v, target_s: float, rows_cap: int = 4096):
+    """Time the oracle on sampled query rows of a few heads, growing the sample
+    until it takes about target_s seconds (bounded).  Returns a dict."""
+    import oracle
+    nthreads = oracle.default_threads()
+    heads = list(range(min(4, w.B * w.H)))
+    count = 8
+    while True:
+        rows = _inputs.sample_rows(w.N, count, w.seed)
+        t0 = time.perf_counter()
+        oracle.attention_rows(q, k, v, w.causal, w.scale, rows=rows, heads=heads,
+                              nthreads=nthreads)
+        dt = time.perf_counter() - t0
+        if dt >= target_s or count >= rows_cap or count >= w.N:
+            break
+        grow = max(2.0, min(8.0, target_s / max(dt, 1e-3)))
+        count = min(rows_cap, w.N, int(count * grow))
+    flops = oracle_sample_flops(w, rows, len(heads))
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+            "seconds": dt, "rows": rows, "heads": heads,
+            "sample": f"{len(rows)} query rows (boundary rows + seeded uniform draws) x "
+                      f"{len(heads)} heads of {w.name}; FLOPs = 4*d*(allowed keys) per row"}
+
+
+# ---------------------------------------------------------------------------
+# Arms
+# ---------------------------------------------------------------------------
+def run_reference(args, w):
+    """The oracle as it stands, timed on the host cores: every step evaluates a
+    fixed sample of query rows, sized so the whole run ends within minutes."""
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    q, k, v = _inputs.workload_inputs(w)
+    per_step = min(args.ref_step_seconds, args.ref_budget_seconds / (args.steps + args.warmup))
+    probe = time_oracle(w, q, k, v, target_s=per_step)   # sizes the sample; first warm-up
+    rows, heads, nthreads = probe.pop("rows"), probe.pop("heads"), probe["cores"]
+    flops = oracle_sample_flops(w, rows, len(heads))
+    for _ in range(max(0, args.warmup - 1)):
+        oracle.attention_rows(q, k, v, w.causal, w.scale, rows=rows, heads=heads,
+                              nthreads=nthreads)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.attention_rows(q, k, v, w.causal, w.scale, rows=rows, heads=heads,
+                              nthreads=nthreads)
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    value = flops / (ms * 1e-3) / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                         "sample": probe["sample"] + " per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, world):
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+            "scale": w.scale, "seed": w.seed, "inputs": "bf16; " + (
+                "Q,K ~ N(0,16), V ~ U(-1,1)" if w.v_dist == "uniform" else "Q,K,V ~ N(0,1)"),
+            "per_rank": "one independent batch per rank (seed + 1000*rank)",
+            "parallelism": f"dp{world}" if world > 1 else "single GPU",
+            "l2": ("inputs larger than L2 (q,k,v %.0f MB per step)" % (
+                3 * 2 * w.B * w.H * w.N * w.d / 1e6))
+            if 3 * 2 * w.B * w.H * w.N * w.d > L2_BYTES else "L2 flushed between steps"}
+
+
+def run_cuda(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import exact_attention_127_b200 as attn
+
+    rank, local, world = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    attn.load_library()
+
+    q, k, v = _inputs.make_qkv(w.B, w.H, w.N, w.d, rank_seed(w.seed, rank), w.qk_std, w.v_dist)
+    qd, kd, vd = (t.to(dev) for t in (q, k, v))
+    o = torch.empty_like(qd)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    flush = None
+    big_enough = 3 * qd.numel() * 2 > L2_BYTES
+    if not big_enough:
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        if flush is not None:
+            flush.fill_(1.0)   # evict L2 between timed iterations
+        attn.attn_fwd(qd, kd, vd, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    if attn.device_status(reset=True, stream=stream) != 0:
+        raise RuntimeError("kernel reported a device-side error during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            if flush is not None:
+                flush.fill_(1.0)
+            starts[i].record(stream)
+            attn.attn_fwd(qd, kd, vd, causal=w.causal, scale=w.scale, out=o, lse=lse,
+                          stream=stream)
+            ends[i].record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    launches = args.steps
+    kernel_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = starts[0].elapsed_time(ends[-1])
+    ms_step = total_ms / args.steps
+    ms_kernel = sum(kernel_ms) / len(kernel_ms)
+    status = attn.device_status(reset=True, stream=stream)
+    if status != 0:
+        raise RuntimeError(f"kernel reported device status {status}")
+
+    # ---- end to end: host (pinned) buffers through the C ABI host entry point
+    qp, kp, vp = (t.pin_memory() for t in (q, k, v))
+    op = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    lp = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
+    ws = torch.empty(attn.host_workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    for _ in range(min(2, args.warmup)):
+        attn.attn_fwd_host(qp, kp, vp, w.causal, w.scale, out=op, lse=lp, workspace=ws,
+                           device=dev, stream=stream, synchronize=True)
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        attn.attn_fwd_host(qp, kp, vp, w.causal, w.scale, out=op, lse=lp, workspace=ws,
+                           device=dev, stream=stream, synchronize=False)
+    e1.record(stream)
+    stream.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if attn.device_status(reset=True, stream=stream) != 0:
+        raise RuntimeError("kernel reported a device-side error in the e2e leg")
+
+    ms_max, kern_max, e2e_max = reduce_max([ms_step, ms_kernel, e2e_ms], dev)
+
+    flops = w.flops()
+    value = aggregate_value(flops, world, ms_max)
+    line = None
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        achieved = flops / (kern_max * 1e-3) / 1e12
+        traffic = load_traffic(w.name)
+        clocks = sampler.summary()
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": config_of(w, world),
+            "roofline": {
+                "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                "traffic": traffic,
+                "peak_source": f"{peak_src} bf16 dense matmul, burst (MEASURED_PEAKS.json)"
+                if peak_src == "measured" else "fallback 1.59 PFLOP/s",
+                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                "frac_of_datasheet_2250": achieved / DATASHEET_BF16_TFLOPS,
+                "kernel": KERNEL_NAME, "kernel_ms": kern_max,
+                "algorithmic_flops_per_launch": flops,
+                "compulsory_bytes_per_launch": w.compulsory_bytes(),
+            },
+            "e2e": {"value": aggregate_value(flops, world, e2e_max), "unit": UNIT,
+                    "ms_per_step": e2e_max,
+                    "h2d_bytes_per_step": 3 * q.numel() * 2,
+                    "d2h_bytes_per_step": q.numel() * 2 + w.B * w.H * w.N * 4,
+                    "path": "attn_fwd_host (pinned host buffers, copies + kernel on one stream)"},
+            "gpu_launches": launches,
+            "clocks": clocks,
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = time_oracle(w, q, k, v, target_s=args.cpu_seconds)
+            cpu.pop("rows")
+            cpu.pop("heads")
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=_inputs.HEADLINE, choices=_inputs.WORKLOAD_ORDER)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=2.0)
+    ap.add_argument("--ref-budget-seconds", type=float, default=150.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override B of the workload (smaller cases for profiler captures)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.steps < 1:
+        ap.error("--steps must be >= 1")
+    w = _inputs.WORKLOADS[args.workload]
+    if args.batch is not None:
+        import dataclasses
+        w = dataclasses.replace(w, B=args.batch, name=f"{w.name}@B{args.batch}")
+    _, _, world = dist_env()
+    if world != args.gpus:
+        sys.stderr.write(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE\n")
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_cuda(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -78,7 +78,7 @@ struct Cfg {
     static constexpr int Q_OFF = 0;
     static constexpr int RING_OFF = 2 * TILE_BYTES;
     static constexpr int BAR_OFF = RING_OFF + NSTAGE * TILE_BYTES;
-    static constexpr int NUM_BARS = 2 + 2 * NSTAGE + 6 + 1;
+    static constexpr int NUM_BARS = 2 + 2 * NSTAGE + 8 + 1;
     static constexpr int MISC_OFF = BAR_OFF + 8 * NUM_BARS;
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
     // TMEM columns: S/P of tile t at 128*t, O of tile t at 256 + D*t
@@ -141,11 +141,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_attn_status, 0, code); }
 
-/* Bounded wait for the phase of parity `parity` of an mbarrier.  Returns false
- * when another warp raised the abort flag, or after the limit (then it records
- * the timeout and raises the flag itself). */
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag) {
-    if (mbar_try(bar, parity)) return true;
+/* Slow path of mbar_wait. */
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag) {
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 0; it < WAIT_MAX_ITERS; ++it) {
         if (mbar_try(bar, parity)) return true;
@@ -157,6 +154,14 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile u
     record_error(ATTN_ERR_TIMEOUT);
     *abort_flag = 1u;
     return false;
+}
+
+/* Bounded wait for the phase of parity `parity` of an mbarrier.  Returns false
+ * when another warp raised the abort flag, or after the limit (then it records
+ * the timeout and raises the flag itself). */
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag) {
+    if (mbar_try(bar, parity)) return true;
+    return mbar_wait_slow(bar, parity, abort_flag);
 }
 
 /* Bounded wait that ignores the abort flag: used on the abort path to let the
@@ -210,13 +215,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+/* The MMA statements carry no memory clobber: they touch no memory the compiler
+ * tracks, and as volatile asm they stay ordered with the (clobbering) waits,
+ * fences and commits around them. */
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                        uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
@@ -224,8 +231,7 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -234,10 +240,61 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
                  : "memory");
 }
 
+/* S = Q K^T for one 128x128 tile: D/16 MMAs with K = 16.  a0 / b0 describe
+ * the first 16 columns of Q and K; k-step kk starts (kk/4) swizzle atoms plus
+ * (kk%4)*32 bytes further, which only moves the start-address field. */
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc) {
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = static_cast<uint64_t>(((kk >> 2) * CHUNK_BYTES + (kk & 3) * 32) >> 4);
+        mma_ss(d_tmem, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
+    }
+}
+
+/* O += P V for keys [64*half, 64*half + 64) of one block: 4 MMAs with K = 16.
+ * P is bf16 in TMEM (keys 2c, 2c+1 in column c); b0 describes V's first 16
+ * keys (MN-major: 16 keys = 2048 bytes further per k-step). */
+__device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, uint64_t b0,
+                                              uint32_t idesc, uint32_t acc_first, int half) {
+#pragma unroll
+    for (int i = 0; i < BLOCK_N / 32; ++i) {
+        const int kk = half * (BLOCK_N / 32) + i;
+        const uint64_t off = static_cast<uint64_t>((kk * 16 * 128) >> 4);
+        mma_ts(d_tmem, p_tmem + kk * 8, b0 + off, idesc, (i > 0) ? 1u : acc_first);
+    }
+}
+
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+/* Packed pairs of fp32 (one 64-bit register pair) for the sm_100 f32x2 pipes. */
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
 }
 
 /* Two fp32 -> one bf16x2 word, round to nearest even; `lo` in bits 0-15. */
@@ -388,7 +445,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint32_t bar_s_full0 = bars + 16 + 16 * NSTAGE;      // [2]
     const uint32_t bar_p_ready0 = bar_s_full0 + 16;            // [2]
     const uint32_t bar_o_full0 = bar_p_ready0 + 16;            // [2]
-    const uint32_t bar_drain = bar_o_full0 + 16;
+    const uint32_t bar_p_half0 = bar_o_full0 + 16;             // [2]
+    const uint32_t bar_drain = bar_p_half0 + 16;
     uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::MISC_OFF);
     volatile uint32_t* const abort_flag = reinterpret_cast<volatile uint32_t*>(base_ptr + C::MISC_OFF + 4);
 
@@ -406,6 +464,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             mbar_init(bar_s_full0 + 8 * t, 1);
             mbar_init(bar_p_ready0 + 8 * t, BLOCK_M);   // every softmax thread of the tile
             mbar_init(bar_o_full0 + 8 * t, 1);
+            mbar_init(bar_p_half0 + 8 * t, BLOCK_M);    // first half of P_t stored
         }
         mbar_init(bar_drain, 1);
         *abort_flag = 0u;
@@ -482,33 +541,20 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16(BLOCK_M, BLOCK_N, false);
             constexpr uint32_t IDESC_PV = idesc_bf16(BLOCK_M, D, true);
-            const uint32_t s_col[2] = {C::S_COL0, C::S_COL1};
-            const uint32_t o_col[2] = {C::O_COL0, C::O_COL1};
+            constexpr uint64_t SLOT_STEP = TILE >> 4;       // descriptor units per ring slot
+            const uint32_t ts0 = tmem + C::S_COL0, ts1 = tmem + C::S_COL1;
+            const uint32_t to0 = tmem + C::O_COL0, to1 = tmem + C::O_COL1;
+            const uint64_t qd0 = sdesc_sw128(sQ[0], 16, 1024);
+            const uint64_t qd1 = sdesc_sw128(sQ[1], 16, 1024);
+            const uint64_t kd_base = sdesc_sw128(sRing, 16, 1024);             // K-major
+            const uint64_t vd_base = sdesc_sw128(sRing, CHUNK_BYTES, 1024);    // MN-major
+            const uint32_t bs0 = bar_s_full0, bs1 = bar_s_full0 + 8;
+            const uint32_t bh0 = bar_p_half0, bh1 = bar_p_half0 + 8;
+            const uint32_t bp0 = bar_p_ready0, bp1 = bar_p_ready0 + 8;
+            const uint32_t bo0 = bar_o_full0, bo1 = bar_o_full0 + 8;
             uint32_t it = 0;
-            uint32_t pr[2] = {0, 0};   // p_ready phases consumed per tile
+            uint32_t pr0 = 0, pr1 = 0;   // p_half / p_ready phases consumed per tile
             int local = 0;
-
-            // S_t = Q_t K^T for the K block in ring slot `slot`
-            auto issue_s = [&](int t, int slot) {
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32;
-                    const uint64_t a = sdesc_sw128(sQ[t] + koff, 16, 1024);
-                    const uint64_t b = sdesc_sw128(sRing + slot * TILE + koff, 16, 1024);
-                    mma_ss(tmem + s_col[t], a, b, IDESC_S, kk > 0 ? 1u : 0u);
-                }
-            };
-            // O_t (+)= P_t V for the V block in ring slot `slot`; P_t is bf16 in TMEM
-            auto issue_pv = [&](int t, int slot, bool acc) {
-#pragma unroll
-                for (int kk = 0; kk < BLOCK_N / 16; ++kk) {
-                    const uint64_t b = sdesc_sw128(sRing + slot * TILE + kk * 16 * 128,
-                                                   CHUNK_BYTES, 1024);
-                    mma_ts(tmem + o_col[t], tmem + s_col[t] + kk * 8, b, IDESC_PV,
-                           (acc || kk > 0) ? 1u : 0u);
-                }
-            };
-
             bool aborted = false;
             for (int r = 0; !aborted; ++r) {
                 const int idx = unit_index(r);
@@ -520,43 +566,53 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tc_fence_after();
                 // K_0
                 {
-                    const int ks = it % NSTAGE;
+                    const uint32_t ks = it % NSTAGE;
                     if (!mbar_wait(bar_kv_full(ks), (it / NSTAGE) & 1u, abort_flag)) { aborted = true; break; }
                     tc_fence_after();
-                    if (n0 > 0) { issue_s(0, ks); mma_commit(bar_s_full0); }
-                    if (n1 > 0) { issue_s(1, ks); mma_commit(bar_s_full0 + 8); }
+                    const uint64_t kd = kd_base + ks * SLOT_STEP;
+                    if (n0 > 0) { issue_qk<D>(ts0, qd0, kd, IDESC_S); mma_commit(bs0); }
+                    if (n1 > 0) { issue_qk<D>(ts1, qd1, kd, IDESC_S); mma_commit(bs1); }
                     if (nmax == 1) mma_commit(bar_q_empty);
                     mma_commit(bar_kv_empty(ks));
                     ++it;
                 }
                 for (int j = 0; j < nmax; ++j) {
-                    const int vs = it % NSTAGE;
+                    const uint32_t vs = it % NSTAGE;
                     if (!mbar_wait(bar_kv_full(vs), (it / NSTAGE) & 1u, abort_flag)) { aborted = true; break; }
                     tc_fence_after();
                     ++it;
+                    const uint64_t vd = vd_base + vs * SLOT_STEP;
+                    const uint32_t acc = j > 0 ? 1u : 0u;
                     const bool has_next = j + 1 < nmax;
-                    const int ks = it % NSTAGE;
+                    const uint32_t ks = it % NSTAGE;
+                    const uint64_t kd = kd_base + ks * SLOT_STEP;
                     bool k_ready = false;
                     if (j < n0) {
-                        if (!mbar_wait(bar_p_ready0, pr[0] & 1u, abort_flag)) { aborted = true; break; }
-                        ++pr[0];
+                        if (!mbar_wait(bh0, pr0 & 1u, abort_flag)) { aborted = true; break; }
                         tc_fence_after();
-                        issue_pv(0, vs, j > 0);
-                        if (j == n0 - 1) mma_commit(bar_o_full0);
+                        issue_pv_half(to0, ts0, vd, IDESC_PV, acc, 0);
+                        if (!mbar_wait(bp0, pr0 & 1u, abort_flag)) { aborted = true; break; }
+                        ++pr0;
+                        tc_fence_after();
+                        issue_pv_half(to0, ts0, vd, IDESC_PV, 1u, 1);
+                        if (j == n0 - 1) mma_commit(bo0);
                     }
                     if (j + 1 < n0) {
                         if (!mbar_wait(bar_kv_full(ks), (it / NSTAGE) & 1u, abort_flag)) { aborted = true; break; }
                         tc_fence_after();
                         k_ready = true;
-                        issue_s(0, ks);
-                        mma_commit(bar_s_full0);
+                        issue_qk<D>(ts0, qd0, kd, IDESC_S);
+                        mma_commit(bs0);
                     }
                     if (j < n1) {
-                        if (!mbar_wait(bar_p_ready0 + 8, pr[1] & 1u, abort_flag)) { aborted = true; break; }
-                        ++pr[1];
+                        if (!mbar_wait(bh1, pr1 & 1u, abort_flag)) { aborted = true; break; }
                         tc_fence_after();
-                        issue_pv(1, vs, j > 0);
-                        if (j == n1 - 1) mma_commit(bar_o_full0 + 8);
+                        issue_pv_half(to1, ts1, vd, IDESC_PV, acc, 0);
+                        if (!mbar_wait(bp1, pr1 & 1u, abort_flag)) { aborted = true; break; }
+                        ++pr1;
+                        tc_fence_after();
+                        issue_pv_half(to1, ts1, vd, IDESC_PV, 1u, 1);
+                        if (j == n1 - 1) mma_commit(bo1);
                     }
                     mma_commit(bar_kv_empty(vs));
                     if (has_next) {
@@ -564,7 +620,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                             if (!mbar_wait(bar_kv_full(ks), (it / NSTAGE) & 1u, abort_flag)) { aborted = true; break; }
                             tc_fence_after();
                         }
-                        if (j + 1 < n1) { issue_s(1, ks); mma_commit(bar_s_full0 + 8); }
+                        if (j + 1 < n1) { issue_qk<D>(ts1, qd1, kd, IDESC_S); mma_commit(bs1); }
                         if (j + 1 == nmax - 1) mma_commit(bar_q_empty);
                         mma_commit(bar_kv_empty(ks));
                         ++it;
@@ -587,6 +643,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t o_addr = lane_base + (t ? C::O_COL1 : C::O_COL0);
         const uint32_t bar_s = bar_s_full0 + 8 * t;
         const uint32_t bar_p = bar_p_ready0 + 8 * t;
+        const uint32_t bar_ph = bar_p_half0 + 8 * t;
         const uint32_t bar_o = bar_o_full0 + 8 * t;
         const float c = p.scale_log2;
         uint32_t sph = 0, oph = 0;
@@ -621,9 +678,18 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     for (int cc = 0; cc < BLOCK_N; ++cc)
                         if (cc >= tail) s[cc] = -INFINITY;
                 }
-                float mx = s[0];
+                // row max: four independent chains of three-input max
+                float m4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-                for (int cc = 1; cc < BLOCK_N; ++cc) mx = fmaxf(mx, s[cc]);
+                for (int cc = 4; cc < BLOCK_N - 4; cc += 8) {
+                    m4[0] = fmax3f(m4[0], s[cc], s[cc + 1]);
+                    m4[1] = fmax3f(m4[1], s[cc + 2], s[cc + 3]);
+                    m4[2] = fmax3f(m4[2], s[cc + 4], s[cc + 5]);
+                    m4[3] = fmax3f(m4[3], s[cc + 6], s[cc + 7]);
+                }
+                m4[0] = fmax3f(m4[0], s[BLOCK_N - 4], s[BLOCK_N - 3]);
+                m4[1] = fmax3f(m4[1], s[BLOCK_N - 2], s[BLOCK_N - 1]);
+                const float mx = fmax3f(m4[0], m4[1], fmaxf(m4[2], m4[3]));
                 const float mb = mx * c;               // block max, log2 units
                 const bool need = mb > m_ref + TAU;
                 float alpha = 1.0f;
@@ -632,23 +698,40 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     l *= alpha;
                     m_ref = mb;
                 }
+                // O_acc needs the factor alpha before P_j V_j lands on it.  That is
+                // rare with lazy rescaling, so a warp that needs it stores all of
+                // P first (the scores are dead by then) and hands P over after
+                // the rescale; otherwise P goes over in two halves so the first
+                // half of P V starts while the second half is computed.
+                const bool warp_rescale = j > 0 && __any_sync(0xffffffffu, need);
                 const float neg_m = (m_ref == -INFINITY) ? 0.0f : -m_ref;
-                uint32_t pk[BLOCK_N / 2];
-                float sum0 = 0.0f, sum1 = 0.0f;
+                const uint64_t c2 = f2pack(c, c);
+                const uint64_t nm2 = f2pack(neg_m, neg_m);
+                float sum_a = 0.0f, sum_b = 0.0f;
 #pragma unroll
-                for (int cc = 0; cc < BLOCK_N / 2; ++cc) {
-                    const float p0 = ex2(fmaf(s[2 * cc], c, neg_m));
-                    const float p1 = ex2(fmaf(s[2 * cc + 1], c, neg_m));
-                    sum0 += p0;
-                    sum1 += p1;
-                    pk[cc] = pack_bf16(p0, p1);
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t pk[BLOCK_N / 4];
+#pragma unroll
+                    for (int k = 0; k < BLOCK_N / 4; ++k) {
+                        const int cc = half * (BLOCK_N / 2) + 2 * k;
+                        float x0, x1;
+                        f2unpack(ffma2(f2pack(s[cc], s[cc + 1]), c2, nm2), x0, x1);
+                        const float p0 = ex2(x0);
+                        const float p1 = ex2(x1);
+                        sum_a += p0;
+                        sum_b += p1;
+                        pk[k] = pack_bf16(p0, p1);
+                    }
+                    tmem_st32(s_addr + half * (BLOCK_N / 4), pk);
+                    if (!warp_rescale) {
+                        tmem_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(half ? bar_p : bar_ph);
+                    }
                 }
-                l += sum0 + sum1;
-                tmem_st32(s_addr, pk);
-                tmem_st32(s_addr + 32, pk + 32);
-                if (j > 0 && __any_sync(0xffffffffu, need)) {
-                    // rescale this row of O_acc in TMEM (PV of block j-1 has
-                    // completed: the commit that released S_j covers it)
+                if (warp_rescale) {
+                    // PV of block j-1 has completed: the commit that released S_j
+                    // covers it, so O_acc is stable here
 #pragma unroll
                     for (int ch = 0; ch < D / 32; ++ch) {
                         uint32_t ov[32];
@@ -658,10 +741,12 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                             ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
                         tmem_st32(o_addr + ch * 32, ov);
                     }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(bar_ph);
+                    mbar_arrive(bar_p);
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar_p);
+                l += sum_a + sum_b;
             }
             if (!ok) break;
             ok = mbar_wait(bar_o, oph & 1u, abort_flag);

@@ -36,7 +36,10 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     tmp = LIB + ".tmp"
     cmd = [nvcc_path(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), SRC, "-o", tmp]
-    res = subprocess.run(cmd, capture_output=True, text=True)
+    try:
+        res = subprocess.run(cmd, capture_output=True, text=True, timeout=900)
+    except subprocess.TimeoutExpired:
+        raise RuntimeError("nvcc timed out after 900 s:\n" + " ".join(cmd))
     if res.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + res.stdout + res.stderr)
     os.replace(tmp, LIB)

@@ -74,10 +74,10 @@ template <int D>
 struct Cfg {
     static constexpr int TILE_BYTES = BLOCK_M * D * 2;   // 128 rows x D bf16
     static constexpr int CHUNKS = D / CHUNK_ELEMS;       // swizzle atoms along d
-    static constexpr int NSTAGE = (D == 128) ? 4 : 8;    // K/V ring slots
+    static constexpr int NSTAGE = (D == 128) ? 2 : 4;    // ring stages, each K_j then V_j
     static constexpr int Q_OFF = 0;
     static constexpr int RING_OFF = 2 * TILE_BYTES;
-    static constexpr int BAR_OFF = RING_OFF + NSTAGE * TILE_BYTES;
+    static constexpr int BAR_OFF = RING_OFF + 2 * NSTAGE * TILE_BYTES;
     static constexpr int NUM_BARS = 2 + 2 * NSTAGE + 8 + 1;
     static constexpr int MISC_OFF = BAR_OFF + 8 * NUM_BARS;
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
@@ -297,6 +297,51 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
     return r;
 }
 
+__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+/* 2^x for a pair of values on the FMA/ALU pipes, to relieve the MUFU unit.
+ * Range reduction (Cody-Waite style): x = n + f with n = round(x), obtained by
+ * adding and subtracting 1.5 * 2^23 in fp32, and f in [-1/2, 1/2].  2^f is the
+ * degree-3 polynomial with minimax relative error on [-1/2, 1/2] (Remez
+ * exchange; coefficients and the fit in fit_exp2_poly.py next to this file;
+ * max relative error 7.5e-5, far below the bf16 rounding of P).  2^n is
+ * applied by adding n to the exponent field: the low mantissa bits of
+ * x + 1.5 * 2^23 hold n, so shifting its bit pattern left by 23 yields n << 23.
+ * x is clamped at -125 so the exponent stays normal (2^-125 is negligible next
+ * to a row whose largest term is >= 1). */
+constexpr float EXP2_ROUND = 12582912.0f;          // 1.5 * 2^23
+constexpr float EXP2_C0 = 9.999280572e-01f;
+constexpr float EXP2_C1 = 6.932609677e-01f;
+constexpr float EXP2_C2 = 2.426111251e-01f;
+constexpr float EXP2_C3 = 5.517166853e-02f;
+
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& p0, float& p1) {
+    const uint64_t x = f2pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+    const uint64_t rnd = f2pack(EXP2_ROUND, EXP2_ROUND);
+    const uint64_t t = fadd2(x, rnd);
+    const uint64_t f = fsub2(x, fsub2(t, rnd));
+    uint64_t q = ffma2(f2pack(EXP2_C3, EXP2_C3), f, f2pack(EXP2_C2, EXP2_C2));
+    q = ffma2(q, f, f2pack(EXP2_C1, EXP2_C1));
+    q = ffma2(q, f, f2pack(EXP2_C0, EXP2_C0));
+    float q0, q1, t0, t1;
+    f2unpack(q, q0, q1);
+    f2unpack(t, t0, t1);
+    p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+    p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
+/* Which column pairs of a score row take the polynomial (bit k%8 of the mask
+ * for pair k); the rest use the MUFU ex2.  3 of 8 pairs balances the MUFU and
+ * FMA pipes for a 128-column block. */
+#ifndef ATTN_EXP2_POLY_MASK
+#define ATTN_EXP2_POLY_MASK 0x00u
+#endif
+constexpr uint32_t EXP2_POLY_MASK = ATTN_EXP2_POLY_MASK;
+
 /* Two fp32 -> one bf16x2 word, round to nearest even; `lo` in bits 0-15. */
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     uint32_t r;
@@ -368,6 +413,19 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* v) {
           "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
           "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
           "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+/* tcgen05.st of 16 consecutive 32-bit columns into this thread's TMEM lane. */
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {"
+        "%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16"
+        "};"
+        :
+        : "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]),
+          "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]),
+          "r"(v[13]), "r"(v[14]), "r"(v[15])
         : "memory");
 }
 
@@ -486,6 +544,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+
     if (warp == LOAD_WARP) {
         /* ---------------- TMA producer ---------------- */
         if (lane == 0) {
@@ -506,21 +565,21 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                         tma_load_3d(&tm_q, sQ[t] + c * CHUNK_BYTES, bar_q_full, c * CHUNK_ELEMS,
                                     u.pair * UNIT_ROWS + t * BLOCK_M, u.bh);
                 const int nmax = u.n[0] > u.n[1] ? u.n[0] : u.n[1];
-                for (int j = 0; j < nmax && !aborted; ++j) {
-                    for (int kv = 0; kv < 2; ++kv) {
-                        const int s = it % NSTAGE;
-                        const uint32_t use = it / NSTAGE;
-                        if (!mbar_wait(bar_kv_empty(s), (use & 1u) ^ 1u, abort_flag)) {
-                            aborted = true;
-                            break;
-                        }
-                        mbar_arrive_expect_tx(bar_kv_full(s), TILE);
-                        const CUtensorMap* m = kv ? &tm_v : &tm_k;
-                        for (int c = 0; c < C::CHUNKS; ++c)
-                            tma_load_3d(m, sRing + s * TILE + c * CHUNK_BYTES, bar_kv_full(s),
-                                        c * CHUNK_ELEMS, j * BLOCK_N, u.bh);
-                        ++it;
+                for (int j = 0; j < nmax; ++j) {
+                    // one ring stage holds K_j and V_j, filled and released together
+                    const int s = it % NSTAGE;
+                    const uint32_t use = it / NSTAGE;
+                    if (!mbar_wait(bar_kv_empty(s), (use & 1u) ^ 1u, abort_flag)) {
+                        aborted = true;
+                        break;
                     }
+                    mbar_arrive_expect_tx(bar_kv_full(s), 2 * TILE);
+                    for (int kv = 0; kv < 2; ++kv)
+                        for (int c = 0; c < C::CHUNKS; ++c)
+                            tma_load_3d(kv ? &tm_v : &tm_k,
+                                        sRing + (2 * s + kv) * TILE + c * CHUNK_BYTES,
+                                        bar_kv_full(s), c * CHUNK_ELEMS, j * BLOCK_N, u.bh);
+                    ++it;
                 }
                 ++local;
                 if (aborted) break;
@@ -537,7 +596,14 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         __syncwarp();
     } else if (warp == MMA_WARP) {
-        /* ---------------- MMA issuer ---------------- */
+        /* ---------------- MMA issuer ----------------
+         * Tensor-core order per K/V block j, one thread:
+         *   P0_j V_j, S0_{j+1}, P1_j V_j, S1_{j+1}
+         * so each tile's softmax of block j+1 overlaps the other tile's GEMMs.
+         * S_t(j+1) overwrites the TMEM columns that hold P_t(j); the tensor
+         * core runs one thread's MMAs in order, so P_t(j) V_j reads P first.
+         * Waits on TMA barriers need no tcgen05 fence (no tcgen05 op precedes
+         * their arrival); waits on softmax barriers do. */
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16(BLOCK_M, BLOCK_N, false);
             constexpr uint32_t IDESC_PV = idesc_bf16(BLOCK_M, D, true);
@@ -546,8 +612,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             const uint32_t to0 = tmem + C::O_COL0, to1 = tmem + C::O_COL1;
             const uint64_t qd0 = sdesc_sw128(sQ[0], 16, 1024);
             const uint64_t qd1 = sdesc_sw128(sQ[1], 16, 1024);
-            const uint64_t kd_base = sdesc_sw128(sRing, 16, 1024);             // K-major
-            const uint64_t vd_base = sdesc_sw128(sRing, CHUNK_BYTES, 1024);    // MN-major
+            const uint64_t kd_base = sdesc_sw128(sRing, 16, 1024);                    // K-major
+            const uint64_t vd_base = sdesc_sw128(sRing + TILE, CHUNK_BYTES, 1024);    // MN-major
             const uint32_t bs0 = bar_s_full0, bs1 = bar_s_full0 + 8;
             const uint32_t bh0 = bar_p_half0, bh1 = bar_p_half0 + 8;
             const uint32_t bp0 = bar_p_ready0, bp1 = bar_p_ready0 + 8;
@@ -563,30 +629,22 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const int n0 = u.n[0], n1 = u.n[1];
                 const int nmax = n0 > n1 ? n0 : n1;
                 if (!mbar_wait(bar_q_full, local & 1, abort_flag)) { aborted = true; break; }
-                tc_fence_after();
-                // K_0
+                // block 0: S0_0, S1_0
                 {
-                    const uint32_t ks = it % NSTAGE;
-                    if (!mbar_wait(bar_kv_full(ks), (it / NSTAGE) & 1u, abort_flag)) { aborted = true; break; }
-                    tc_fence_after();
-                    const uint64_t kd = kd_base + ks * SLOT_STEP;
+                    const uint32_t st = it % NSTAGE;
+                    if (!mbar_wait(bar_kv_full(st), (it / NSTAGE) & 1u, abort_flag)) { aborted = true; break; }
+                    const uint64_t kd = kd_base + 2 * st * SLOT_STEP;
                     if (n0 > 0) { issue_qk<D>(ts0, qd0, kd, IDESC_S); mma_commit(bs0); }
                     if (n1 > 0) { issue_qk<D>(ts1, qd1, kd, IDESC_S); mma_commit(bs1); }
                     if (nmax == 1) mma_commit(bar_q_empty);
-                    mma_commit(bar_kv_empty(ks));
-                    ++it;
                 }
                 for (int j = 0; j < nmax; ++j) {
-                    const uint32_t vs = it % NSTAGE;
-                    if (!mbar_wait(bar_kv_full(vs), (it / NSTAGE) & 1u, abort_flag)) { aborted = true; break; }
-                    tc_fence_after();
-                    ++it;
-                    const uint64_t vd = vd_base + vs * SLOT_STEP;
+                    const uint32_t st = it % NSTAGE;                 // stage of block j
+                    const uint64_t vd = vd_base + 2 * st * SLOT_STEP;
                     const uint32_t acc = j > 0 ? 1u : 0u;
                     const bool has_next = j + 1 < nmax;
-                    const uint32_t ks = it % NSTAGE;
-                    const uint64_t kd = kd_base + ks * SLOT_STEP;
-                    bool k_ready = false;
+                    const uint32_t nx = it + 1;                      // ring position of block j+1
+                    const uint64_t kd = kd_base + 2 * (nx % NSTAGE) * SLOT_STEP;
                     if (j < n0) {
                         if (!mbar_wait(bh0, pr0 & 1u, abort_flag)) { aborted = true; break; }
                         tc_fence_after();
@@ -597,13 +655,12 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                         issue_pv_half(to0, ts0, vd, IDESC_PV, 1u, 1);
                         if (j == n0 - 1) mma_commit(bo0);
                     }
-                    if (j + 1 < n0) {
-                        if (!mbar_wait(bar_kv_full(ks), (it / NSTAGE) & 1u, abort_flag)) { aborted = true; break; }
-                        tc_fence_after();
-                        k_ready = true;
-                        issue_qk<D>(ts0, qd0, kd, IDESC_S);
-                        mma_commit(bs0);
+                    if (has_next &&
+                        !mbar_wait(bar_kv_full(nx % NSTAGE), (nx / NSTAGE) & 1u, abort_flag)) {
+                        aborted = true;
+                        break;
                     }
+                    if (j + 1 < n0) { issue_qk<D>(ts0, qd0, kd, IDESC_S); mma_commit(bs0); }
                     if (j < n1) {
                         if (!mbar_wait(bh1, pr1 & 1u, abort_flag)) { aborted = true; break; }
                         tc_fence_after();
@@ -614,17 +671,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                         issue_pv_half(to1, ts1, vd, IDESC_PV, 1u, 1);
                         if (j == n1 - 1) mma_commit(bo1);
                     }
-                    mma_commit(bar_kv_empty(vs));
-                    if (has_next) {
-                        if (!k_ready) {
-                            if (!mbar_wait(bar_kv_full(ks), (it / NSTAGE) & 1u, abort_flag)) { aborted = true; break; }
-                            tc_fence_after();
-                        }
-                        if (j + 1 < n1) { issue_qk<D>(ts1, qd1, kd, IDESC_S); mma_commit(bs1); }
-                        if (j + 1 == nmax - 1) mma_commit(bar_q_empty);
-                        mma_commit(bar_kv_empty(ks));
-                        ++it;
-                    }
+                    mma_commit(bar_kv_empty(st));                    // K_j and V_j read
+                    ++it;
+                    if (j + 1 < n1) { issue_qk<D>(ts1, qd1, kd, IDESC_S); mma_commit(bs1); }
+                    if (j + 1 == nmax - 1) mma_commit(bar_q_empty);  // last S of the unit issued
                 }
                 ++local;
             }
@@ -709,21 +759,27 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const uint64_t nm2 = f2pack(neg_m, neg_m);
                 float sum_a = 0.0f, sum_b = 0.0f;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t pk[BLOCK_N / 4];
+                for (int qtr = 0; qtr < 4; ++qtr) {
+                    const int half = qtr >> 1;
+                    uint32_t pk[BLOCK_N / 8];
 #pragma unroll
-                    for (int k = 0; k < BLOCK_N / 4; ++k) {
-                        const int cc = half * (BLOCK_N / 2) + 2 * k;
+                    for (int k = 0; k < BLOCK_N / 8; ++k) {
+                        const int cc = qtr * (BLOCK_N / 4) + 2 * k;
                         float x0, x1;
                         f2unpack(ffma2(f2pack(s[cc], s[cc + 1]), c2, nm2), x0, x1);
-                        const float p0 = ex2(x0);
-                        const float p1 = ex2(x1);
+                        float p0, p1;
+                        if ((EXP2_POLY_MASK >> ((qtr * (BLOCK_N / 8) + k) & 7)) & 1u) {
+                            exp2_poly_pair(x0, x1, p0, p1);
+                        } else {
+                            p0 = ex2(x0);
+                            p1 = ex2(x1);
+                        }
                         sum_a += p0;
                         sum_b += p1;
                         pk[k] = pack_bf16(p0, p1);
                     }
-                    tmem_st32(s_addr + half * (BLOCK_N / 4), pk);
-                    if (!warp_rescale) {
+                    tmem_st16(s_addr + qtr * (BLOCK_N / 8), pk);
+                    if (!warp_rescale && (qtr & 1)) {
                         tmem_wait_st();
                         tc_fence_before();
                         mbar_arrive(half ? bar_p : bar_ph);

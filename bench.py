@@ -187,28 +187,30 @@ def oracle_sample_flops(w, rows, n_heads):
     return 4.0 * w.d * keys * n_heads
 
 
-def time_oracle(w, q, k, v, target_s: float, rows_cap: int = 4096):
-    """Time the oracle on sampled query rows of a few heads, growing the sample
-    until it takes about target_s seconds (bounded).  Returns a dict."""
+def time_oracle(w, q, k, v, target_s: float, max_heads: int = 16):
+    """Time the oracle on sampled query rows of the first few heads, growing the
+    row sample until one evaluation takes about target_s seconds (bounded by
+    N rows per head).  Returns a dict (value in the bench's unit)."""
     import oracle
     nthreads = oracle.default_threads()
-    heads = list(range(min(4, w.B * w.H)))
-    count = 8
+    heads = list(range(min(max_heads, w.B * w.H)))
+    count = 4
     while True:
         rows = _inputs.sample_rows(w.N, count, w.seed)
         t0 = time.perf_counter()
         oracle.attention_rows(q, k, v, w.causal, w.scale, rows=rows, heads=heads,
                               nthreads=nthreads)
         dt = time.perf_counter() - t0
-        if dt >= target_s or count >= rows_cap or count >= w.N:
+        if dt >= 0.5 * target_s or count >= w.N:
             break
-        grow = max(2.0, min(8.0, target_s / max(dt, 1e-3)))
-        count = min(rows_cap, w.N, int(count * grow))
+        grow = max(2.0, min(16.0, target_s / max(dt, 1e-3)))
+        count = min(w.N, int(count * grow))
     flops = oracle_sample_flops(w, rows, len(heads))
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": nthreads, "kind": "oracle",
             "seconds": dt, "rows": rows, "heads": heads,
             "sample": f"{len(rows)} query rows (boundary rows + seeded uniform draws) x "
-                      f"{len(heads)} heads of {w.name}; FLOPs = 4*d*(allowed keys) per row"}
+                      f"{len(heads)} heads of {w.name}; FLOPs = 4*d*(allowed keys) per row; "
+                      f"includes widening the heads' bf16 inputs to fp64"}
 
 
 # ---------------------------------------------------------------------------
@@ -223,7 +225,7 @@ def run_reference(args, w):
     import oracle
     q, k, v = _inputs.workload_inputs(w)
     per_step = min(args.ref_step_seconds, args.ref_budget_seconds / (args.steps + args.warmup))
-    probe = time_oracle(w, q, k, v, target_s=per_step)   # sizes the sample; first warm-up
+    probe = time_oracle(w, q, k, v, target_s=per_step, max_heads=4)   # sizes the sample
     rows, heads, nthreads = probe.pop("rows"), probe.pop("heads"), probe["cores"]
     flops = oracle_sample_flops(w, rows, len(heads))
     for _ in range(max(0, args.warmup - 1)):

@@ -729,17 +729,16 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                         if (cc >= tail) s[cc] = -INFINITY;
                 }
                 // row max: four independent chains of three-input max
-                float m4[4] = {s[0], s[1], s[2], s[3]};
+                float m8[8];
 #pragma unroll
-                for (int cc = 4; cc < BLOCK_N - 4; cc += 8) {
-                    m4[0] = fmax3f(m4[0], s[cc], s[cc + 1]);
-                    m4[1] = fmax3f(m4[1], s[cc + 2], s[cc + 3]);
-                    m4[2] = fmax3f(m4[2], s[cc + 4], s[cc + 5]);
-                    m4[3] = fmax3f(m4[3], s[cc + 6], s[cc + 7]);
+                for (int i = 0; i < 8; ++i) m8[i] = fmaxf(s[i], s[i + 8]);
+#pragma unroll
+                for (int cc = 16; cc < BLOCK_N; cc += 16) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) m8[i] = fmax3f(m8[i], s[cc + i], s[cc + 8 + i]);
                 }
-                m4[0] = fmax3f(m4[0], s[BLOCK_N - 4], s[BLOCK_N - 3]);
-                m4[1] = fmax3f(m4[1], s[BLOCK_N - 2], s[BLOCK_N - 1]);
-                const float mx = fmax3f(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+                const float mx = fmax3f(fmax3f(m8[0], m8[1], m8[2]), fmax3f(m8[3], m8[4], m8[5]),
+                                        fmaxf(m8[6], m8[7]));
                 const float mb = mx * c;               // block max, log2 units
                 const bool need = mb > m_ref + TAU;
                 float alpha = 1.0f;

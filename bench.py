@@ -399,12 +399,107 @@ def run_cuda(args, w):
     return 0
 
 
+DECODE_METRIC = "split-K/V decode attention GB/s (K/V cache bytes read / time)"
+
+
+def run_decode(args, w):
+    """One step = one attn_decode call (split kernel + combine kernel) over a
+    batch of one query row per head against N cached keys; HBM-bound."""
+    import torch
+    import torch.distributed as dist
+
+    import exact_attention_127_b200 as attn
+
+    rank, local, world = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    attn.load_library()
+    q, k, v = _inputs.make_decode_qkv(w.B, w.H, w.N, w.d, rank_seed(w.seed, rank))
+    qd, kd, vd = (t.to(dev) for t in (q, k, v))
+    o = torch.empty_like(qd)
+    lse = torch.empty((w.B, w.H), dtype=torch.float32, device=dev)
+    ws = torch.empty(attn.decode_workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(dev)
+    flush = None
+    if 2 * kd.numel() * 2 <= L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            attn.attn_decode(qd, kd, vd, scale=w.scale, out=o, lse=lse, workspace=ws, stream=stream)
+    stream.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            if flush is not None:
+                flush.fill_(1.0)
+            starts[i].record(stream)
+            attn.attn_decode(qd, kd, vd, scale=w.scale, out=o, lse=lse, workspace=ws, stream=stream)
+            ends[i].record(stream)
+    stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    if attn.device_status(reset=True, stream=stream) != 0:
+        raise RuntimeError("device-side error in the decode kernels")
+    step_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
+    (ms_max,) = reduce_max([step_ms], dev)
+    nbytes = w.compulsory_bytes()
+    value = nbytes * world / (ms_max * 1e-3) / 1e9
+    line = None
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        line = {
+            "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                       "queries_per_head": 1, "scale": w.scale, "seed": w.seed,
+                       "parallelism": f"dp{world}" if world > 1 else "single GPU",
+                       "l2": "K/V cache larger than L2" if flush is None else "L2 flushed"},
+            "roofline": {"bound": "hbm", "achieved": value / world, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": value / world / peaks["hbm_gbs"],
+                         "traffic": load_traffic(w.name),
+                         "peak_source": f"{peak_src} HBM copy (MEASURED_PEAKS.json)",
+                         "kernel": "decode_split_kernel + decode_combine_kernel (one call)",
+                         "compulsory_bytes_per_launch": nbytes},
+            "e2e": None, "gpu_launches": 2 * args.steps, "clocks": sampler.summary(),
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            heads = list(range(min(16, w.B * w.H)))
+            t0 = time.perf_counter()
+            oracle.attention_qk(q.reshape(w.B * w.H, 1, 1, w.d)[heads],
+                                k.reshape(w.B * w.H, 1, w.N, w.d)[heads],
+                                v.reshape(w.B * w.H, 1, w.N, w.d)[heads], w.scale)
+            dt = time.perf_counter() - t0
+            cpu_bytes = nbytes * len(heads) / (w.B * w.H)
+            line["cpu_baseline"] = {"value": cpu_bytes / dt / 1e9, "unit": "GB/s",
+                                    "cores": oracle.default_threads(), "kind": "oracle",
+                                    "sample": f"{len(heads)} heads of {w.name}"}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=_inputs.HEADLINE, choices=_inputs.WORKLOAD_ORDER)
+    ap.add_argument("--workload", default=_inputs.HEADLINE,
+                    choices=_inputs.WORKLOAD_ORDER + sorted(_inputs.DECODE_WORKLOADS))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -418,6 +513,12 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.steps < 1:
         ap.error("--steps must be >= 1")
+    if args.workload in _inputs.DECODE_WORKLOADS:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the decode mode has no "
+                              "reference arm; the oracle is timed in its cpu_baseline"}))
+            return 0
+        return run_decode(args, _inputs.DECODE_WORKLOADS[args.workload])
     w = _inputs.WORKLOADS[args.workload]
     if args.batch is not None:
         import dataclasses

@@ -52,6 +52,13 @@ def load_library():
     lib.attn_fwd_host_workspace_bytes.restype = ctypes.c_size_t
     lib.attn_device_status.argtypes = [vp, c_int]
     lib.attn_device_status.restype = c_int
+    lib.attn_decode_workspace_bytes.argtypes = [i64, i64, i64, i64]
+    lib.attn_decode_workspace_bytes.restype = ctypes.c_size_t
+    lib.attn_decode.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, ctypes.c_float, vp,
+                                ctypes.c_size_t, vp]
+    lib.attn_decode.restype = c_int
+    lib.attn_fwd_test_wait_timeout.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
+    lib.attn_fwd_test_wait_timeout.restype = c_int
     lib.attn_status_str.argtypes = [c_int]
     lib.attn_status_str.restype = ctypes.c_char_p
     lib.attn_version.argtypes = []
@@ -174,6 +181,47 @@ def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: boo
                 stream.synchronize()
             else:
                 torch.cuda.synchronize(device)
+    return out, lse
+
+
+def decode_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(load_library().attn_decode_workspace_bytes(B, H, N, d))
+
+
+def attn_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None,
+                out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                workspace: torch.Tensor | None = None, stream=None):
+    """One query row per head against N cached keys (split-K/V decode).
+
+    q: bf16 CUDA [B, H, 1, d] (or [B, H, d]); k, v: bf16 CUDA [B, H, N, d].
+    Returns (o bf16 [B, H, 1, d] shaped like q, lse fp32 [B, H]).
+    """
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise ValueError(f"{name} must be a bf16 CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if k.dim() != 4 or k.shape != v.shape:
+        raise ValueError("k and v must share one [B, H, N, d] shape")
+    B, H, N, d = k.shape
+    if tuple(q.shape) not in ((B, H, 1, d), (B, H, d)):
+        raise ValueError("q must be [B, H, 1, d] or [B, H, d]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(decode_workspace_bytes(B, H, N, d), 1), dtype=torch.uint8,
+                                device=q.device)
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        rc = lib.attn_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             lse.data_ptr(), B, H, N, d, float(scale), workspace.data_ptr(),
+                             workspace.numel(), _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_decode")
     return out, lse
 
 

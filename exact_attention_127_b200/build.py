@@ -11,6 +11,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC = os.path.join(PKG, "csrc", "attn_fwd_sm100.cu")
+SOURCES = [SRC, os.path.join(PKG, "csrc", "attn_decode.cu")]
 HDR = os.path.join(ROOT, "include", "attn_fwd.h")
 LIB = os.path.join(PKG, "libattn127.so")
 
@@ -31,11 +32,11 @@ def nvcc_path() -> str:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    newest = max(os.path.getmtime(SRC), os.path.getmtime(HDR))
+    newest = max(max(os.path.getmtime(f) for f in SOURCES), os.path.getmtime(HDR))
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest:
         return LIB
     tmp = LIB + ".tmp"
-    cmd = [nvcc_path(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), SRC, "-o", tmp]
+    cmd = [nvcc_path(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), *SOURCES, "-o", tmp]
     try:
         res = subprocess.run(cmd, capture_output=True, text=True, timeout=900)
     except subprocess.TimeoutExpired:

@@ -65,7 +65,8 @@ constexpr int TMEM_COLS = 512;
 constexpr int CHUNK_ELEMS = 64;                     // one 128-byte swizzle atom of bf16
 constexpr int CHUNK_BYTES = BLOCK_M * 128;          // 128 rows x 128 bytes
 constexpr float TAU = 8.0f;           // lazy-rescale threshold, log2 units
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s: a correct run never waits 1 ms
+constexpr uint64_t TEST_WAIT_LIMIT_NS = 20000000ull; // 20 ms, for the timeout test hook
 constexpr uint32_t WAIT_MAX_ITERS = 1u << 28;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float LOG2E = 1.4426950408889634f;
@@ -97,6 +98,8 @@ struct FwdParams {
     int nkv;        // ceil(N / 128)
     int n_units;    // BH * n_pairs
     float scale_log2;  // scale * log2(e)
+    uint64_t wait_limit_ns;  // bound on every mbarrier wait
+    int withhold_kv;         // test hook: the producer never loads K/V, so waits run out
 };
 
 __device__ int g_attn_status = 0;
@@ -142,13 +145,14 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_attn_status, 0, code); }
 
 /* Slow path of mbar_wait. */
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag) {
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                            uint64_t limit_ns) {
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 0; it < WAIT_MAX_ITERS; ++it) {
         if (mbar_try(bar, parity)) return true;
         if ((it & 63u) == 63u) {
             if (*abort_flag) return false;
-            if (globaltimer() - t0 > WAIT_LIMIT_NS) break;
+            if (globaltimer() - t0 > limit_ns) break;
         }
     }
     record_error(ATTN_ERR_TIMEOUT);
@@ -159,18 +163,19 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volat
 /* Bounded wait for the phase of parity `parity` of an mbarrier.  Returns false
  * when another warp raised the abort flag, or after the limit (then it records
  * the timeout and raises the flag itself). */
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                          uint64_t limit_ns) {
     if (mbar_try(bar, parity)) return true;
-    return mbar_wait_slow(bar, parity, abort_flag);
+    return mbar_wait_slow(bar, parity, abort_flag, limit_ns);
 }
 
 /* Bounded wait that ignores the abort flag: used on the abort path to let the
  * CTA's own copies and MMAs in flight land before it exits. */
-__device__ __noinline__ void mbar_drain_wait(uint32_t bar, uint32_t parity) {
+__device__ __noinline__ void mbar_drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 0; it < WAIT_MAX_ITERS; ++it) {
         if (mbar_try(bar, parity)) return;
-        if ((it & 63u) == 63u && globaltimer() - t0 > WAIT_LIMIT_NS) return;
+        if ((it & 63u) == 63u && globaltimer() - t0 > limit_ns) return;
     }
 }
 
@@ -510,6 +515,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint64_t wlim = p.wait_limit_ns;
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q_full, 1);
@@ -555,7 +561,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const int idx = unit_index(r);
                 if (idx >= p.n_units) break;
                 const Unit u = unit_at<CAUSAL>(idx, p);
-                if (local > 0 && !mbar_wait(bar_q_empty, (local - 1) & 1, abort_flag)) {
+                if (local > 0 && !mbar_wait(bar_q_empty, (local - 1) & 1, abort_flag, wlim)) {
                     aborted = true;
                     break;
                 }
@@ -564,12 +570,12 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     for (int c = 0; c < C::CHUNKS; ++c)
                         tma_load_3d(&tm_q, sQ[t] + c * CHUNK_BYTES, bar_q_full, c * CHUNK_ELEMS,
                                     u.pair * UNIT_ROWS + t * BLOCK_M, u.bh);
-                const int nmax = u.n[0] > u.n[1] ? u.n[0] : u.n[1];
+                const int nmax = p.withhold_kv ? 0 : (u.n[0] > u.n[1] ? u.n[0] : u.n[1]);
                 for (int j = 0; j < nmax; ++j) {
                     // one ring stage holds K_j and V_j, filled and released together
                     const int s = it % NSTAGE;
                     const uint32_t use = it / NSTAGE;
-                    if (!mbar_wait(bar_kv_empty(s), (use & 1u) ^ 1u, abort_flag)) {
+                    if (!mbar_wait(bar_kv_empty(s), (use & 1u) ^ 1u, abort_flag, wlim)) {
                         aborted = true;
                         break;
                     }
@@ -586,11 +592,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             if (aborted) {
                 /* let this CTA's copies in flight land before the CTA exits */
-                if (local > 0) mbar_drain_wait(bar_q_full, (local - 1) & 1);
+                if (local > 0) mbar_drain_wait(bar_q_full, (local - 1) & 1, wlim);
                 const uint32_t n_back = it < (uint32_t)NSTAGE ? it : (uint32_t)NSTAGE;
                 for (uint32_t b = 1; b <= n_back; ++b) {
                     const uint32_t i = it - b;
-                    mbar_drain_wait(bar_kv_full(i % NSTAGE), (i / NSTAGE) & 1u);
+                    mbar_drain_wait(bar_kv_full(i % NSTAGE), (i / NSTAGE) & 1u, wlim);
                 }
             }
         }
@@ -628,11 +634,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const Unit u = unit_at<CAUSAL>(idx, p);
                 const int n0 = u.n[0], n1 = u.n[1];
                 const int nmax = n0 > n1 ? n0 : n1;
-                if (!mbar_wait(bar_q_full, local & 1, abort_flag)) { aborted = true; break; }
+                if (!mbar_wait(bar_q_full, local & 1, abort_flag, wlim)) { aborted = true; break; }
                 // block 0: S0_0, S1_0
                 {
                     const uint32_t st = it % NSTAGE;
-                    if (!mbar_wait(bar_kv_full(st), (it / NSTAGE) & 1u, abort_flag)) { aborted = true; break; }
+                    if (!mbar_wait(bar_kv_full(st), (it / NSTAGE) & 1u, abort_flag, wlim)) { aborted = true; break; }
                     const uint64_t kd = kd_base + 2 * st * SLOT_STEP;
                     if (n0 > 0) { issue_qk<D>(ts0, qd0, kd, IDESC_S); mma_commit(bs0); }
                     if (n1 > 0) { issue_qk<D>(ts1, qd1, kd, IDESC_S); mma_commit(bs1); }
@@ -646,26 +652,26 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const uint32_t nx = it + 1;                      // ring position of block j+1
                     const uint64_t kd = kd_base + 2 * (nx % NSTAGE) * SLOT_STEP;
                     if (j < n0) {
-                        if (!mbar_wait(bh0, pr0 & 1u, abort_flag)) { aborted = true; break; }
+                        if (!mbar_wait(bh0, pr0 & 1u, abort_flag, wlim)) { aborted = true; break; }
                         tc_fence_after();
                         issue_pv_half(to0, ts0, vd, IDESC_PV, acc, 0);
-                        if (!mbar_wait(bp0, pr0 & 1u, abort_flag)) { aborted = true; break; }
+                        if (!mbar_wait(bp0, pr0 & 1u, abort_flag, wlim)) { aborted = true; break; }
                         ++pr0;
                         tc_fence_after();
                         issue_pv_half(to0, ts0, vd, IDESC_PV, 1u, 1);
                         if (j == n0 - 1) mma_commit(bo0);
                     }
                     if (has_next &&
-                        !mbar_wait(bar_kv_full(nx % NSTAGE), (nx / NSTAGE) & 1u, abort_flag)) {
+                        !mbar_wait(bar_kv_full(nx % NSTAGE), (nx / NSTAGE) & 1u, abort_flag, wlim)) {
                         aborted = true;
                         break;
                     }
                     if (j + 1 < n0) { issue_qk<D>(ts0, qd0, kd, IDESC_S); mma_commit(bs0); }
                     if (j < n1) {
-                        if (!mbar_wait(bh1, pr1 & 1u, abort_flag)) { aborted = true; break; }
+                        if (!mbar_wait(bh1, pr1 & 1u, abort_flag, wlim)) { aborted = true; break; }
                         tc_fence_after();
                         issue_pv_half(to1, ts1, vd, IDESC_PV, acc, 0);
-                        if (!mbar_wait(bp1, pr1 & 1u, abort_flag)) { aborted = true; break; }
+                        if (!mbar_wait(bp1, pr1 & 1u, abort_flag, wlim)) { aborted = true; break; }
                         ++pr1;
                         tc_fence_after();
                         issue_pv_half(to1, ts1, vd, IDESC_PV, 1u, 1);
@@ -680,7 +686,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             /* all MMAs this thread issued have completed once this phase lands */
             mma_commit(bar_drain);
-            mbar_drain_wait(bar_drain, 0);
+            mbar_drain_wait(bar_drain, 0, wlim);
         }
         __syncwarp();
     } else {
@@ -710,7 +716,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             float l = 0.0f;            // running sum of 2^(c*s - m_ref)
             bool ok = true;
             for (int j = 0; j < n; ++j) {
-                ok = mbar_wait(bar_s, sph & 1u, abort_flag);
+                ok = mbar_wait(bar_s, sph & 1u, abort_flag, wlim);
                 ++sph;
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
@@ -804,7 +810,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                 l += sum_a + sum_b;
             }
             if (!ok) break;
-            ok = mbar_wait(bar_o, oph & 1u, abort_flag);
+            ok = mbar_wait(bar_o, oph & 1u, abort_flag, wlim);
             ++oph;
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
@@ -965,12 +971,10 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
     return ATTN_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
-             int64_t H, int64_t N, int64_t d, int causal, float scale, void* stream) {
+/* The forward call behind attn_fwd and the timeout test hook. */
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+             int64_t H, int64_t N, int64_t d, int causal, float scale, void* stream,
+             uint64_t wait_limit_ns, int withhold_kv) {
     bool empty = false;
     int st = validate_shape(B, H, N, d, scale, &empty);
     if (st != ATTN_OK || empty) return st;
@@ -1006,10 +1010,26 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
     prm.nkv = static_cast<int>((N + BLOCK_N - 1) / BLOCK_N);
     prm.n_units = prm.BH * prm.n_pairs;
     prm.scale_log2 = scale * LOG2E;
+    prm.wait_limit_ns = wait_limit_ns;
+    prm.withhold_kv = withhold_kv;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (d == 64)
         return causal ? launch<64, true>(mq, mk, mv, prm, di, s) : launch<64, false>(mq, mk, mv, prm, di, s);
     return causal ? launch<128, true>(mq, mk, mv, prm, di, s) : launch<128, false>(mq, mk, mv, prm, di, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+             int64_t H, int64_t N, int64_t d, int causal, float scale, void* stream) {
+    return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, stream, WAIT_LIMIT_NS, 0);
+}
+
+int attn_fwd_test_wait_timeout(const void* q, const void* k, const void* v, void* o, float* lse,
+                               int64_t B, int64_t H, int64_t N, int64_t d, void* stream) {
+    return fwd_impl(q, k, v, o, lse, B, H, N, d, 0, 0.125f, stream, TEST_WAIT_LIMIT_NS, 1);
 }
 
 static size_t align256(size_t x) { return (x + 255u) & ~static_cast<size_t>(255u); }

@@ -89,6 +89,47 @@ def make_qkv(B: int, H: int, N: int, d: int, seed: int, qk_std: float = 1.0,
     return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
 
 
+@dataclass(frozen=True)
+class DecodeWorkload:
+    """One new query row per head against N cached keys (decode)."""
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def flops(self) -> float:
+        return 4.0 * self.B * self.H * self.N * self.d
+
+    def compulsory_bytes(self) -> int:
+        """K and V read once (the cache), q read and o written (bf16), lse written."""
+        return 2 * 2 * self.B * self.H * self.N * self.d + 2 * 2 * self.B * self.H * self.d \
+            + 4 * self.B * self.H
+
+
+DECODE_WORKLOADS = {
+    "decode_b16h16_n8192_d128": DecodeWorkload("decode_b16h16_n8192_d128", 16, 16, 8192, 128, 5),
+    "decode_b4h16_n32768_d128": DecodeWorkload("decode_b4h16_n32768_d128", 4, 16, 32768, 128, 6),
+    "decode_b32h32_n4096_d64": DecodeWorkload("decode_b32h32_n4096_d64", 32, 32, 4096, 64, 7),
+}
+
+
+def make_decode_qkv(B: int, H: int, N: int, d: int, seed: int):
+    """Seeded bf16 CPU tensors: q [B, H, 1, d] drawn first, then k and v
+    [B, H, N, d], all N(0, 1), each rounded to bf16 (RNE)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    q = torch.randn((B, H, 1, d), generator=g, dtype=torch.float32)
+    k = torch.randn((B, H, N, d), generator=g, dtype=torch.float32)
+    v = torch.randn((B, H, N, d), generator=g, dtype=torch.float32)
+    return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+
 def workload_inputs(w: Workload):
     return make_qkv(w.B, w.H, w.N, w.d, w.seed, w.qk_std, w.v_dist)
 

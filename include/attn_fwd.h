@@ -18,8 +18,9 @@
  *   - Tensors are dense and row-major: q, k, v, o are bf16 [B, H, N, d] with d
  *     contiguous; lse is fp32 [B, H, N].  Q, K and V share one sequence length
  *     N (self-attention; the causal mask is aligned at the top-left corner).
- *   - d must be 64 or 128.  B, H, N >= 1; B*H < 2^31; N < 2^31.  A call with
- *     B*H*N == 0 is not an error: it returns ATTN_OK and launches nothing.
+ *   - d must be 64 or 128.  B, H, N >= 0; B*H < 2^31; N < 2^31 - 512.  A call
+ *     with B*H*N == 0 is not an error: it returns ATTN_OK and launches nothing
+ *     (the pointers may then be NULL).
  *   - scale must be finite and > 0 (1/sqrt(d) is the usual choice).
  *   - Device pointers must be 16-byte aligned (the tensor-memory-accelerator
  *     copies require it).  o and lse must not overlap q, k, v or each other.
@@ -99,6 +100,45 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
  * cleared afterwards.  Returns ATTN_ERR_CUDA if the word cannot be read.
  */
 int attn_device_status(void* stream, int reset);
+
+/*
+ * attn_decode_workspace_bytes -- device workspace attn_decode needs for a shape
+ * (the per-split partial results).  Returns 0 for invalid or empty shapes.
+ */
+size_t attn_decode_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
+
+/*
+ * attn_decode -- attention of ONE new query row per head against N cached keys
+ * and values (decoding; "GPU 学习日报 Day 21", section 9 and FAQ Q5), with the
+ * key range split across thread blocks and the partial results merged by the
+ * online-softmax rule ("Q31：FlashAttention 为什么快", follow-up 3).
+ *   q   : device, bf16 [B, H, d] (a [B, H, 1, d] tensor), read only.
+ *   k, v: device, bf16 [B, H, N, d], read only.
+ *   o   : device, bf16 [B, H, d], written: softmax(scale * q K^T) V (no mask:
+ *         the query sees every key).
+ *   lse : device, fp32 [B, H], written: ln sum_j exp(scale * q . k_j).
+ *   workspace: device scratch of at least attn_decode_workspace_bytes bytes,
+ *         256-byte aligned, owned by the caller; its contents on entry are
+ *         ignored.  Calls that overlap on the GPU must not share it.
+ * Two kernels are enqueued on `stream` (split, then combine).  Same d, scale,
+ * alignment and error conventions as attn_fwd; ATTN_ERR_WORKSPACE when the
+ * workspace is missing, misaligned or too small.
+ */
+int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse,
+                int64_t B, int64_t H, int64_t N, int64_t d, float scale,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * attn_fwd_test_wait_timeout -- test hook for failure detection, not an
+ * attention call.  Launches the forward kernel (non-causal, same arguments and
+ * checks as attn_fwd) with the producer told never to load K and V, and with
+ * every bounded wait limited to 20 ms.  The waits run out, the kernel records
+ * ATTN_ERR_TIMEOUT in the device status word, frees its tensor memory and
+ * exits; o and lse are left unspecified.  No fault or hang is involved and
+ * the context stays usable.  Read the outcome with attn_device_status.
+ */
+int attn_fwd_test_wait_timeout(const void* q, const void* k, const void* v, void* o, float* lse,
+                               int64_t B, int64_t H, int64_t N, int64_t d, void* stream);
 
 /* attn_status_str -- a static, human-readable string for a status code. */
 const char* attn_status_str(int status);

@@ -19,6 +19,8 @@ marshals arrays.  Sources of each definition (FlashAttention teaching pages):
 * ``softmax_two_pass`` / ``online_softmax`` -- the vector softmax of sections
   5.1/5.2 and practice exercise 2 (online vs two-pass).
 * ``prob_row`` -- the probability row P_i of ``attention_rows``.
+* ``attention_qk`` -- the same definition for Nq query rows against Nk keys
+  (non-causal; the decode case Nq = 1 of page 2, section 9 and FAQ Q5).
 """
 from __future__ import annotations
 
@@ -50,9 +52,11 @@ def _lib():
                                                      dp, dp, ctypes.c_int]
         lib.oracle_attention_prob_row.argtypes = [dp, dp, dp, i64, i64, i64, ctypes.c_int,
                                                   ctypes.c_double, i64, i64, dp]
+        lib.oracle_attention_rows_qk.argtypes = [dp, dp, dp, i64, i64, i64, i64, ctypes.c_double,
+                                                 i64p, i64p, i64, dp, dp, ctypes.c_int]
         for fn in (lib.oracle_softmax_two_pass, lib.oracle_online_softmax,
                    lib.oracle_attention_rows, lib.oracle_attention_rows_online,
-                   lib.oracle_attention_prob_row):
+                   lib.oracle_attention_prob_row, lib.oracle_attention_rows_qk):
             fn.restype = ctypes.c_int
         _LIB = lib
     return _LIB
@@ -176,6 +180,36 @@ def attention(q, k, v, causal: bool, scale: float, nthreads: int | None = None):
     B, H, N, d = tuple(q.shape)
     O, L = attention_rows(q, k, v, causal, scale, nthreads=nthreads)
     return O.reshape(B, H, N, d), L.reshape(B, H, N)
+
+
+def attention_qk(q, k, v, scale: float, heads=None, nthreads: int | None = None):
+    """Non-causal attention of every query row of q [B, H, Nq, d] against the
+    keys/values k, v [B, H, Nk, d] (decode: Nq = 1).  Returns
+    (O [len(heads), Nq, d] fp64, LSE [len(heads), Nq] fp64)."""
+    B, H, Nq, d = tuple(q.shape)
+    if tuple(k.shape[:2]) != (B, H) or tuple(k.shape) != tuple(v.shape) or k.shape[3] != d:
+        raise ValueError("q [B, H, Nq, d] and k, v [B, H, Nk, d] required")
+    Nk = k.shape[2]
+    BH = B * H
+    heads = list(range(BH)) if heads is None else [int(h) for h in heads]
+    nthreads = default_threads() if nthreads is None else int(nthreads)
+    rows = np.arange(Nq, dtype=np.int64)
+    zeros = np.zeros(Nq, dtype=np.int64)
+    O = np.empty((len(heads), Nq, d), dtype=np.float64)
+    L = np.empty((len(heads), Nq), dtype=np.float64)
+    qf, kf, vf = q.reshape(BH, Nq, d), k.reshape(BH, Nk, d), v.reshape(BH, Nk, d)
+    for n, bh in enumerate(heads):
+        qh, kh, vh = _f64(qf[bh]), _f64(kf[bh]), _f64(vf[bh])
+        o = np.empty((Nq, d), dtype=np.float64)
+        lse = np.empty(Nq, dtype=np.float64)
+        rc = _lib().oracle_attention_rows_qk(_dptr(qh), _dptr(kh), _dptr(vh), 1, Nq, Nk, d,
+                                             float(scale), _iptr(zeros), _iptr(rows), Nq,
+                                             _dptr(o), _dptr(lse), nthreads)
+        if rc != 0:
+            raise ValueError(f"oracle failed with status {rc}")
+        O[n] = o
+        L[n] = lse
+    return O, L
 
 
 def prob_row(q, k, v, causal: bool, scale: float, head: int, row: int) -> np.ndarray:

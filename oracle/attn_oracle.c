@@ -165,7 +165,7 @@ static void attention_row_online(const double* qi, const double* K, const double
 /* ------------------------------------------------------------------------ */
 typedef struct {
     const double *q, *k, *v;
-    int64_t N, d;
+    int64_t Nq, N, d;   /* query rows and key rows per head */
     int causal;
     double scale;
     int64_t block;          /* 0 = three-step definition, > 0 = online recurrence */
@@ -180,9 +180,10 @@ static void* run_rows(void* arg) {
     double* s = (double*)malloc(sizeof(double) * (size_t)(jb->N > 0 ? jb->N : 1));
     if (!s) { jb->status = -2; return NULL; }
     const int64_t head = jb->N * jb->d;
+    const int64_t head_q = jb->Nq * jb->d;
     for (int64_t r = jb->first; r < jb->nrows; r += jb->stride) {
         const int64_t bh = jb->bh_idx[r], i = jb->row_idx[r];
-        const double* qi = jb->q + bh * head + i * jb->d;
+        const double* qi = jb->q + bh * head_q + i * jb->d;
         const double* K = jb->k + bh * head;
         const double* V = jb->v + bh * head;
         if (jb->block > 0)
@@ -197,20 +198,21 @@ static void* run_rows(void* arg) {
 }
 
 static int run_parallel(const double* q, const double* k, const double* v, int64_t BH,
-                        int64_t N, int64_t d, int causal, double scale, int64_t block,
+                        int64_t Nq, int64_t N, int64_t d, int causal, double scale, int64_t block,
                         const int64_t* bh_idx, const int64_t* row_idx, int64_t nrows,
                         double* o_out, double* lse_out, int nthreads) {
     if (!q || !k || !v || !bh_idx || !row_idx || !o_out || !lse_out) return -1;
-    if (BH <= 0 || N <= 0 || d <= 0 || nrows < 0) return -1;
+    if (BH <= 0 || Nq <= 0 || N <= 0 || d <= 0 || nrows < 0) return -1;
+    if (causal && Nq != N) return -1;   /* causal is defined for square attention only */
     for (int64_t r = 0; r < nrows; ++r)
-        if (bh_idx[r] < 0 || bh_idx[r] >= BH || row_idx[r] < 0 || row_idx[r] >= N) return -1;
+        if (bh_idx[r] < 0 || bh_idx[r] >= BH || row_idx[r] < 0 || row_idx[r] >= Nq) return -1;
     if (nthreads < 1) nthreads = 1;
     if (nthreads > 256) nthreads = 256;
     if ((int64_t)nthreads > nrows) nthreads = nrows > 0 ? (int)nrows : 1;
     job_t jobs[256];
     pthread_t th[256];
     for (int t = 0; t < nthreads; ++t) {
-        job_t jb = {q, k, v, N, d, causal, scale, block, bh_idx, row_idx, nrows, t, nthreads,
+        job_t jb = {q, k, v, Nq, N, d, causal, scale, block, bh_idx, row_idx, nrows, t, nthreads,
                     o_out, lse_out, 0};
         jobs[t] = jb;
     }
@@ -237,7 +239,21 @@ int oracle_attention_rows(const double* q, const double* k, const double* v, int
                           int64_t N, int64_t d, int causal, double scale,
                           const int64_t* bh_idx, const int64_t* row_idx, int64_t nrows,
                           double* o_out, double* lse_out, int nthreads) {
-    return run_parallel(q, k, v, BH, N, d, causal, scale, 0, bh_idx, row_idx, nrows,
+    return run_parallel(q, k, v, BH, N, N, d, causal, scale, 0, bh_idx, row_idx, nrows,
+                        o_out, lse_out, nthreads);
+}
+
+/*
+ * Non-causal attention of Nq query rows against Nk key/value rows per head
+ * (the decode case, Nq = 1: one new query attends to every cached key; page 2,
+ * section 9 and FAQ Q5).  q: [BH, Nq, d]; k, v: [BH, Nk, d].  The same
+ * three-step definition per row.
+ */
+int oracle_attention_rows_qk(const double* q, const double* k, const double* v, int64_t BH,
+                             int64_t Nq, int64_t Nk, int64_t d, double scale,
+                             const int64_t* bh_idx, const int64_t* row_idx, int64_t nrows,
+                             double* o_out, double* lse_out, int nthreads) {
+    return run_parallel(q, k, v, BH, Nq, Nk, d, 0, scale, 0, bh_idx, row_idx, nrows,
                         o_out, lse_out, nthreads);
 }
 
@@ -247,7 +263,7 @@ int oracle_attention_rows_online(const double* q, const double* k, const double*
                                  int64_t block, const int64_t* bh_idx, const int64_t* row_idx,
                                  int64_t nrows, double* o_out, double* lse_out, int nthreads) {
     if (block < 1) return -1;
-    return run_parallel(q, k, v, BH, N, d, causal, scale, block, bh_idx, row_idx, nrows,
+    return run_parallel(q, k, v, BH, N, N, d, causal, scale, block, bh_idx, row_idx, nrows,
                         o_out, lse_out, nthreads);
 }
 

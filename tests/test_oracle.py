@@ -299,6 +299,7 @@ def _pins_pass():
             test_key_shift_moves_lse_not_output(causal)
         test_causal_row0_is_v0(5)
         test_single_key_returns_its_value_row(4)
+        test_decode_brute_force(1, 7, 4)
     except AssertionError:
         return False
     return True
@@ -320,9 +321,69 @@ def test_planted_mistakes_are_caught(mutant, tmp_path, monkeypatch):
     real = oracle._lib()
     mut = ctypes.CDLL(str(lib))
     for name in ("oracle_softmax_two_pass", "oracle_online_softmax", "oracle_attention_rows",
-                 "oracle_attention_rows_online", "oracle_attention_prob_row"):
+                 "oracle_attention_rows_online", "oracle_attention_prob_row",
+                 "oracle_attention_rows_qk"):
         getattr(mut, name).argtypes = getattr(real, name).argtypes
         getattr(mut, name).restype = getattr(real, name).restype
     assert _pins_pass()
     monkeypatch.setattr(oracle, "_LIB", mut)
     assert not _pins_pass(), f"planted mistake {mutant!r} went unnoticed"
+
+
+# ---------------------------------------------------------------------------
+# Decode (one query against many keys): attention_qk
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("Nq,Nk,d", [(1, 1, 3), (1, 7, 4), (3, 5, 2), (1, 8, 1)])
+def test_decode_brute_force(Nq, Nk, d):
+    q = _rand((1, 1, Nq, d), 60)
+    k, v = _rand((1, 1, Nk, d), 61), _rand((1, 1, Nk, d), 62)
+    O, L = oracle.attention_qk(q, k, v, 0.6)
+    getcontext().prec = 40
+    for i in range(Nq):
+        e = []
+        for j in range(Nk):
+            s = sum(Decimal(repr(float(q[0, 0, i, c]))) * Decimal(repr(float(k[0, 0, j, c])))
+                    for c in range(d))
+            e.append((Decimal(repr(0.6)) * s).exp())
+        z = sum(e)
+        for c in range(d):
+            ref = float(sum(x * Decimal(repr(float(v[0, 0, j, c]))) for j, x in enumerate(e)) / z)
+            assert abs(O[0, i, c] - ref) < 1e-12
+        assert abs(L[0, i] - float(z.ln())) < 1e-12
+
+
+def test_decode_single_key_and_zero_query():
+    q, k, v = _rand((2, 1, 1, 8), 63), _rand((2, 1, 1, 8), 64), _rand((2, 1, 1, 8), 65)
+    O, L = oracle.attention_qk(q, k, v, 0.4)
+    for h in range(2):
+        assert np.array_equal(O[h, 0], v[h, 0, 0])
+        assert L[h, 0] == pytest.approx(0.4 * float(q[h, 0, 0] @ k[h, 0, 0]), rel=1e-14, abs=1e-14)
+    k2, v2 = _rand((1, 1, 50, 8), 66), _rand((1, 1, 50, 8), 67)
+    O, L = oracle.attention_qk(np.zeros((1, 1, 1, 8)), k2, v2, 0.4)
+    assert np.allclose(O[0, 0], v2[0, 0].mean(axis=0), rtol=0, atol=1e-14)
+    assert L[0, 0] == pytest.approx(math.log(50), rel=1e-14)
+
+
+@pytest.mark.parametrize("split", [1, 17, 64, 99])
+def test_split_and_merge_matches_whole(split):
+    """Q31, follow-up 3 (split K/V, compute the parts, merge) with the merge
+    rule of the online recurrence (page 2, section 5.2): weights e^{LSE_part}."""
+    N = 100
+    q = _rand((1, 2, 1, 16), 68, 2.0)
+    k, v = _rand((1, 2, N, 16), 69, 2.0), _rand((1, 2, N, 16), 70)
+    O, L = oracle.attention_qk(q, k, v, 0.25)
+    O1, L1 = oracle.attention_qk(q, k[:, :, :split], v[:, :, :split], 0.25)
+    O2, L2 = oracle.attention_qk(q, k[:, :, split:], v[:, :, split:], 0.25)
+    M = np.maximum(L1, L2)
+    w1, w2 = np.exp(L1 - M), np.exp(L2 - M)
+    Lm = M + np.log(w1 + w2)
+    Om = (w1[..., None] * O1 + w2[..., None] * O2) / (w1 + w2)[..., None]
+    assert np.max(np.abs(Om - O)) < 1e-13
+    assert np.max(np.abs(Lm - L)) < 1e-13
+
+
+def test_decode_rejects_bad_shapes():
+    with pytest.raises(ValueError):
+        oracle.attention_qk(np.zeros((1, 1, 1, 4)), np.zeros((1, 1, 5, 4)), np.zeros((1, 1, 6, 4)), 1.0)
+    with pytest.raises(ValueError):
+        oracle.attention_qk(np.zeros((1, 1, 1, 4)), np.zeros((1, 2, 5, 4)), np.zeros((1, 2, 5, 4)), 1.0)

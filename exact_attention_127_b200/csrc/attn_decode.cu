@@ -29,6 +29,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "attn_fwd.h"
 
 namespace {
@@ -280,6 +282,62 @@ int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse
     }
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
     return ATTN_OK;
+}
+
+}  // extern "C"
+
+/*
+ * Allocation-free decode.  Some callers cannot allocate device memory
+ * themselves: a plugin or runtime whose host application owns all device
+ * memory through its own pool, or a latency-bound loop that must not call
+ * cudaMalloc (which can synchronise the device) once it is running.  For them
+ * the per-split partial results live in this fixed buffer, part of the
+ * library's own device image.  It is created with the module on every GPU
+ * that loads the library and stays until the process exits.
+ */
+constexpr size_t DECODE_STATIC_SCRATCH_BYTES = size_t(8) << 20;   // 8 MiB
+static __device__ __align__(256) unsigned char g_decode_scratch[DECODE_STATIC_SCRATCH_BYTES];
+
+namespace {
+constexpr int SCRATCH_MAX_DEVICES = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[SCRATCH_MAX_DEVICES] = {};
+
+/* Device address of g_decode_scratch on the current device.  In host code the
+ * array's name only stands in for the symbol, so the address is looked up once
+ * per device (with that device current) and cached. */
+int scratch_address(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return ATTN_ERR_CUDA; }
+    if (dev < 0 || dev >= SCRATCH_MAX_DEVICES) return ATTN_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_ptr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || !ptr) {
+            cudaGetLastError();
+            return ATTN_ERR_CUDA;
+        }
+        g_scratch_ptr[dev] = ptr;
+    }
+    *out = g_scratch_ptr[dev];
+    return ATTN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+size_t attn_decode_noalloc_scratch_bytes(void) { return DECODE_STATIC_SCRATCH_BYTES; }
+
+int attn_decode_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int64_t B, int64_t H, int64_t N, int64_t d, float scale, void* stream) {
+    bool empty = false;
+    int st = decode_validate(B, H, N, d, scale, &empty);
+    if (st != ATTN_OK || empty) return st;
+    if (decode_ws_bytes(B * H, N, d) > DECODE_STATIC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    if ((st = scratch_address(&scratch)) != ATTN_OK) return st;
+    return attn_decode(q, k, v, o, lse, B, H, N, d, scale, scratch, DECODE_STATIC_SCRATCH_BYTES,
+                       stream);
 }
 
 }  // extern "C"

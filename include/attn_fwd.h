@@ -129,6 +129,34 @@ int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse
                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * attn_decode_noalloc -- attn_decode for callers that cannot allocate device
+ * memory.  The pages have no counterpart: this entry point exists for callers
+ * that may not call cudaMalloc themselves, such as a plugin whose host
+ * application owns every device allocation through its own pool, or a
+ * latency-bound loop that must not allocate (cudaMalloc can synchronise the
+ * device) once it runs.  It takes the same arguments as attn_decode minus the
+ * workspace and allocates nothing: the per-split partial results go to a fixed
+ * static device buffer inside the library, attn_decode_noalloc_scratch_bytes()
+ * = 8 MiB, which every GPU that loads the library holds until the process
+ * exits.
+ *   - Shapes whose partials need more than that (attn_decode_workspace_bytes
+ *     > 8 MiB; roughly B*H*splits*(d+2)*4 bytes, e.g. any B*H beyond 16384 at
+ *     d = 128) are rejected with ATTN_ERR_WORKSPACE before anything runs.
+ *   - The buffer's device address is looked up on the first call on each
+ *     device, with that device current; make that first call outside any
+ *     stream capture.
+ *   - Every call shares the one buffer, which keeps the last call's partials.
+ *     Nothing in it has to start at zero (every partial is written before it
+ *     is read), but calls that overlap on the GPU (other streams, other host
+ *     threads) race on it: serialise them.
+ */
+int attn_decode_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int64_t B, int64_t H, int64_t N, int64_t d, float scale, void* stream);
+
+/* attn_decode_noalloc_scratch_bytes -- size of the static buffer above (8 MiB). */
+size_t attn_decode_noalloc_scratch_bytes(void);
+
+/*
  * attn_fwd_test_wait_timeout -- test hook for failure detection, not an
  * attention call.  Launches the forward kernel (non-causal, same arguments and
  * checks as attn_fwd) with the producer told never to load K and V, and with

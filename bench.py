@@ -402,6 +402,67 @@ def run_cuda(args, w):
 DECODE_METRIC = "split-K/V decode attention GB/s (K/V cache bytes read / time)"
 
 
+def run_standard(args, w):
+    """The unfused three-kernel path on a forward workload (context for the
+    fused kernel): same metric (useful TFLOP/s); its roofline is HBM, since the
+    N x N matrices cross device memory four times."""
+    import torch
+
+    import exact_attention_127_b200 as attn
+
+    rank, local, world = dist_env()
+    if world > 1:
+        raise SystemExit("--path standard runs on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    attn.load_library()
+    q, k, v = (t.to(dev) for t in _inputs.workload_inputs(w))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    ws = torch.empty(attn.standard_workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            attn.attn_standard(q, k, v, w.causal, w.scale, out=o, lse=lse, workspace=ws,
+                               stream=stream)
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    sampler.start()
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            attn.attn_standard(q, k, v, w.causal, w.scale, out=o, lse=lse, workspace=ws,
+                               stream=stream)
+    e1.record(stream)
+    stream.synchronize()
+    sampler.stop()
+    if attn.device_status(reset=True, stream=stream) != 0:
+        raise RuntimeError("device-side error in the standard path")
+    ms = e0.elapsed_time(e1) / args.steps
+    Np = (w.N + 127) // 128 * 128
+    nn_bytes = w.B * w.H * Np * Np * (4 + 4 + 2 + 2)    # S written+read (fp32), P written+read
+    nbytes = nn_bytes + w.compulsory_bytes()
+    peaks, peak_src = load_peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": w.flops() / (ms * 1e-3) / 1e12, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "path": "standard: S = scale*QK^T (fp32) -> HBM, softmax -> P (bf16) in place, O = PV",
+        "config": config_of(w, 1),
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "algorithmic_bytes_per_launch": nbytes,
+                     "peak_source": f"{peak_src} HBM copy (MEASURED_PEAKS.json)",
+                     "kernel": "std_qk_kernel + std_softmax_kernel + std_pv_kernel"},
+        "e2e": None, "gpu_launches": 3 * args.steps, "clocks": sampler.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_decode(args, w):
     """One step = one attn_decode call (split kernel + combine kernel) over a
     batch of one query row per head against N cached keys; HBM-bound."""
@@ -506,6 +567,8 @@ def main(argv=None):
     ap.add_argument("--ref-step-seconds", type=float, default=2.0)
     ap.add_argument("--ref-budget-seconds", type=float, default=150.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", default="fused", choices=["fused", "standard"],
+                    help="fused kernel (default) or the unfused three-kernel path for comparison")
     ap.add_argument("--batch", type=int, default=None,
                     help="override B of the workload (smaller cases for profiler captures)")
     args = ap.parse_args(argv)
@@ -528,6 +591,8 @@ def main(argv=None):
         sys.stderr.write(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE\n")
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.path == "standard":
+        return run_standard(args, w)
     return run_cuda(args, w)
 
 

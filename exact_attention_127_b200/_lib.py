@@ -52,6 +52,11 @@ def load_library():
     lib.attn_fwd_host_workspace_bytes.restype = ctypes.c_size_t
     lib.attn_device_status.argtypes = [vp, c_int]
     lib.attn_device_status.restype = c_int
+    lib.attn_standard_workspace_bytes.argtypes = [i64, i64, i64, i64]
+    lib.attn_standard_workspace_bytes.restype = ctypes.c_size_t
+    lib.attn_standard.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, c_int, ctypes.c_float,
+                                  vp, ctypes.c_size_t, vp]
+    lib.attn_standard.restype = c_int
     lib.attn_decode_workspace_bytes.argtypes = [i64, i64, i64, i64]
     lib.attn_decode_workspace_bytes.restype = ctypes.c_size_t
     lib.attn_decode.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, ctypes.c_float, vp,
@@ -181,6 +186,37 @@ def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: boo
                 stream.synchronize()
             else:
                 torch.cuda.synchronize(device)
+    return out, lse
+
+
+def standard_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(load_library().attn_standard_workspace_bytes(B, H, N, d))
+
+
+def attn_standard(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+                  scale: float | None = None, out: torch.Tensor | None = None,
+                  lse: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                  stream=None):
+    """The unfused three-kernel path (S and P through device memory), for
+    comparison with attn_fwd.  Same inputs and outputs as attn_fwd."""
+    _check_inputs(q, k, v, device_expected=True)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(standard_workspace_bytes(B, H, N, d), 1), dtype=torch.uint8,
+                                device=q.device)
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        rc = lib.attn_standard(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                               lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                               workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_standard")
     return out, lse
 
 

@@ -32,7 +32,8 @@ def nvcc_path() -> str:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    newest = max(max(os.path.getmtime(f) for f in SOURCES), os.path.getmtime(HDR))
+    deps = SOURCES + [os.path.join(PKG, "csrc", "attn_standard.cuh"), HDR]
+    newest = max(os.path.getmtime(f) for f in deps)
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest:
         return LIB
     tmp = LIB + ".tmp"

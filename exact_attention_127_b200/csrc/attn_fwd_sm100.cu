@@ -916,11 +916,11 @@ int device_info(int* dev_out, DeviceInfo** info_out) {
 /* 3-D view [B*H][N][d] of a bf16 tensor, box = 64 columns x 128 rows x 1 head,
  * 128-byte swizzle; rows past N read as zeros. */
 int encode_map(EncodeTiledFn fn, CUtensorMap* map, const void* ptr, int64_t BH, int64_t N,
-               int64_t d) {
+               int64_t d, uint32_t box_rows = BLOCK_M) {
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                           static_cast<cuuint64_t>(BH)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(N * d * 2)};
-    cuuint32_t box[3] = {CHUNK_ELEMS, BLOCK_M, 1};
+    cuuint32_t box[3] = {CHUNK_ELEMS, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -969,6 +969,102 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
     kern<<<grid, NUM_THREADS, SMEM, stream>>>(mq, mk, mv, prm);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
     return ATTN_OK;
+}
+
+#include "attn_standard.cuh"
+
+/* The unfused three-kernel path (S and P through device memory), host side. */
+size_t std_ws_bytes(int64_t BH, int64_t N) {
+    const int64_t Np = (N + BLOCK_M - 1) / BLOCK_M * BLOCK_M;
+    return static_cast<size_t>(BH) * Np * Np * sizeof(float);
+}
+
+int std_validate(int64_t B, int64_t H, int64_t N, int64_t d, float scale, bool* empty) {
+    int st = validate_shape(B, H, N, d, scale, empty);
+    if (st != ATTN_OK || *empty) return st;
+    if (N > STD_MAX_N || B * H > 65535) return ATTN_ERR_SHAPE;
+    return ATTN_OK;
+}
+
+template <int D>
+int std_launch(const void* q, const void* k, const void* v, const StdParams& prm,
+               EncodeTiledFn enc, cudaStream_t stream) {
+    CUtensorMap mq, mk, mv, mp;
+    int st;
+    if ((st = encode_map(enc, &mq, q, prm.BH, prm.N, D)) != ATTN_OK) return st;
+    if ((st = encode_map(enc, &mk, k, prm.BH, prm.N, D)) != ATTN_OK) return st;
+    if ((st = encode_map(enc, &mv, v, prm.BH, prm.N, D, STD_PV_KEYS)) != ATTN_OK) return st;
+    {   // P: bf16 over the first half of every fp32 S row (row pitch 4 * Np bytes)
+        const int64_t Np = prm.Np;
+        cuuint64_t dims[3] = {static_cast<cuuint64_t>(Np), static_cast<cuuint64_t>(Np),
+                              static_cast<cuuint64_t>(prm.BH)};
+        cuuint64_t strides[2] = {static_cast<cuuint64_t>(Np * 4),
+                                 static_cast<cuuint64_t>(Np * Np * 4)};
+        cuuint32_t box[3] = {STD_PV_KEYS, BLOCK_M, 1};
+        cuuint32_t estr[3] = {1, 1, 1};
+        if (enc(&mp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, prm.S, dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+            CUDA_SUCCESS)
+            return ATTN_ERR_CUDA;
+    }
+    // kernel 1 keeps at most 3-4 CTAs per SM so their TMEM columns fit
+    const int smem1 = (2 * BLOCK_M * D * 2 > 56 * 1024 ? 2 * BLOCK_M * D * 2 : 56 * 1024) + 2048;
+    constexpr int stage = BLOCK_M * STD_PV_KEYS * 2 + STD_PV_KEYS * D * 2;
+    const int smem3 = STD_PV_STAGES * stage + 16 * STD_PV_STAGES + 64 + 1024;
+    auto k1 = std_qk_kernel<D>;
+    auto k3 = std_pv_kernel<D>;
+    if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1) != cudaSuccess ||
+        cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, smem3) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_LAUNCH;
+    }
+    const unsigned tiles = static_cast<unsigned>(prm.Np / BLOCK_M);
+    k1<<<dim3(tiles, tiles, prm.BH), STD_THREADS, smem1, stream>>>(mq, mk, prm);
+    const int64_t rows = static_cast<int64_t>(prm.BH) * prm.N;
+    if (prm.Np <= STD_SHORT_MAX_NP) {
+        const int64_t per = STD_SOFTMAX_THREADS / 32;
+        std_softmax_short_kernel<<<static_cast<unsigned>((rows + per - 1) / per),
+                                   STD_SOFTMAX_THREADS, 0, stream>>>(prm);
+    } else {
+        std_softmax_kernel<<<static_cast<unsigned>(rows), STD_SOFTMAX_THREADS, 0, stream>>>(prm);
+    }
+    k3<<<dim3(tiles, prm.BH), STD_THREADS, smem3, stream>>>(mp, mv, prm);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+    return ATTN_OK;
+}
+
+int std_impl(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+             int64_t H, int64_t N, int64_t d, int causal, float scale, void* workspace,
+             size_t workspace_bytes, void* stream) {
+    bool empty = false;
+    int st = std_validate(B, H, N, d, scale, &empty);
+    if (st != ATTN_OK || empty) return st;
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
+    const void* ptrs[5] = {q, k, v, o, lse};
+    for (const void* ptr : ptrs)
+        if (reinterpret_cast<uintptr_t>(ptr) & 15u) return ATTN_ERR_ALIGN;
+    const int64_t BH = B * H;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+        workspace_bytes < std_ws_bytes(BH, N))
+        return ATTN_ERR_WORKSPACE;
+    int dev = 0;
+    DeviceInfo* di = nullptr;
+    if ((st = device_info(&dev, &di)) != ATTN_OK) return st;
+    EncodeTiledFn enc = nullptr;
+    if ((st = get_encode(&enc)) != ATTN_OK) return st;
+    StdParams prm;
+    prm.S = static_cast<float*>(workspace);
+    prm.lse = lse;
+    prm.o = static_cast<__nv_bfloat16*>(o);
+    prm.N = static_cast<int>(N);
+    prm.Np = static_cast<int>((N + BLOCK_M - 1) / BLOCK_M * BLOCK_M);
+    prm.BH = static_cast<int>(BH);
+    prm.causal = causal ? 1 : 0;
+    prm.scale = scale;
+    prm.wait_limit_ns = WAIT_LIMIT_NS;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return d == 64 ? std_launch<64>(q, k, v, prm, enc, s) : std_launch<128>(q, k, v, prm, enc, s);
 }
 
 /* The forward call behind attn_fwd and the timeout test hook. */
@@ -1030,6 +1126,19 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
 int attn_fwd_test_wait_timeout(const void* q, const void* k, const void* v, void* o, float* lse,
                                int64_t B, int64_t H, int64_t N, int64_t d, void* stream) {
     return fwd_impl(q, k, v, o, lse, B, H, N, d, 0, 0.125f, stream, TEST_WAIT_LIMIT_NS, 1);
+}
+
+size_t attn_standard_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {
+    bool empty = false;
+    if (std_validate(B, H, N, d, 1.0f, &empty) != ATTN_OK || empty) return 0;
+    return std_ws_bytes(B * H, N);
+}
+
+int attn_standard(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+                  int64_t H, int64_t N, int64_t d, int causal, float scale, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+    return std_impl(q, k, v, o, lse, B, H, N, d, causal, scale, workspace, workspace_bytes,
+                    stream);
 }
 
 static size_t align256(size_t x) { return (x + 255u) & ~static_cast<size_t>(255u); }

@@ -102,6 +102,27 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
 int attn_device_status(void* stream, int reset);
 
 /*
+ * attn_standard_workspace_bytes -- device workspace attn_standard needs: the
+ * N x N score matrix of every head in fp32, rows padded to a multiple of 128
+ * (4 * B * H * Np^2 bytes, Np = N rounded up to 128).  0 for invalid shapes.
+ */
+size_t attn_standard_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
+
+/*
+ * attn_standard -- the same attention computed the standard, unfused way, for
+ * comparison with attn_fwd ("GPU 学习日报 Day 21", sections 3.1 and 4.2: three
+ * kernels, the N x N matrices written to and read back from device memory).
+ * Enqueues on `stream`: S = scale * Q K^T into the workspace (fp32), a row
+ * softmax that writes P (bf16, in place) and LSE, and O = P V.  Same layouts,
+ * outputs and error codes as attn_fwd, plus: N <= 32768, B*H <= 65535, and a
+ * device workspace of at least attn_standard_workspace_bytes (256-byte
+ * aligned, caller-owned, contents ignored on entry).
+ */
+int attn_standard(const void* q, const void* k, const void* v, void* o, float* lse,
+                  int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * attn_decode_workspace_bytes -- device workspace attn_decode needs for a shape
  * (the per-split partial results).  Returns 0 for invalid or empty shapes.
  */

@@ -21,6 +21,10 @@ marshals arrays.  Sources of each definition (FlashAttention teaching pages):
 * ``prob_row`` -- the probability row P_i of ``attention_rows``.
 * ``attention_qk`` -- the same definition for Nq query rows against Nk keys
   (non-causal; the decode case Nq = 1 of page 2, section 9 and FAQ Q5).
+* ``attention_backward`` -- gradients of sum(dO * O) with respect to q, k, v:
+  the chain rule through the three steps, every N x N matrix materialised
+  (the gradients the backward pass recomputes from saved statistics,
+  "science-depth-m4-047" section 3 point (c)).
 """
 from __future__ import annotations
 
@@ -54,9 +58,12 @@ def _lib():
                                                   ctypes.c_double, i64, i64, dp]
         lib.oracle_attention_rows_qk.argtypes = [dp, dp, dp, i64, i64, i64, i64, ctypes.c_double,
                                                  i64p, i64p, i64, dp, dp, ctypes.c_int]
+        lib.oracle_attention_backward.argtypes = [dp, dp, dp, dp, i64, i64, ctypes.c_int,
+                                                  ctypes.c_double, dp, dp, dp, ctypes.c_int]
         for fn in (lib.oracle_softmax_two_pass, lib.oracle_online_softmax,
                    lib.oracle_attention_rows, lib.oracle_attention_rows_online,
-                   lib.oracle_attention_prob_row, lib.oracle_attention_rows_qk):
+                   lib.oracle_attention_prob_row, lib.oracle_attention_rows_qk,
+                   lib.oracle_attention_backward):
             fn.restype = ctypes.c_int
         _LIB = lib
     return _LIB
@@ -210,6 +217,31 @@ def attention_qk(q, k, v, scale: float, heads=None, nthreads: int | None = None)
         O[n] = o
         L[n] = lse
     return O, L
+
+
+def attention_backward(q, k, v, dout, causal: bool, scale: float, heads=None,
+                       nthreads: int | None = None):
+    """(dQ, dK, dV) fp64, each [len(heads), N, d], for the given heads of
+    q, k, v, dout [B, H, N, d]."""
+    shape = tuple(q.shape)
+    if len(shape) != 4 or any(tuple(t.shape) != shape for t in (k, v, dout)):
+        raise ValueError("q, k, v, dout must share one [B, H, N, d] shape")
+    B, H, N, d = shape
+    BH = B * H
+    heads = list(range(BH)) if heads is None else [int(h) for h in heads]
+    nthreads = default_threads() if nthreads is None else int(nthreads)
+    out = [np.empty((len(heads), N, d), dtype=np.float64) for _ in range(3)]
+    flat = [t.reshape(BH, N, d) for t in (q, k, v, dout)]
+    for n, bh in enumerate(heads):
+        qh, kh, vh, oh = (_f64(t[bh]) for t in flat)
+        dq, dk, dv = (np.empty((N, d), dtype=np.float64) for _ in range(3))
+        rc = _lib().oracle_attention_backward(_dptr(qh), _dptr(kh), _dptr(vh), _dptr(oh), N, d,
+                                              int(bool(causal)), float(scale), _dptr(dq),
+                                              _dptr(dk), _dptr(dv), nthreads)
+        if rc != 0:
+            raise ValueError(f"oracle failed with status {rc}")
+        out[0][n], out[1][n], out[2][n] = dq, dk, dv
+    return tuple(out)
 
 
 def prob_row(q, k, v, causal: bool, scale: float, head: int, row: int) -> np.ndarray:

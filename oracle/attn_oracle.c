@@ -24,6 +24,13 @@
  *     is provided as a second, independent function so that the tests can pin
  *     the two against each other (the pages claim exact equality up to
  *     floating-point order: page 2 FAQ Q1; page 1 section 3).
+ *   - The backward pass (page 1, section 3, point (c): gradients recomputed
+ *     from the saved statistics) is checked against the gradients of the same
+ *     definition, written out in fp64 with every N x N matrix materialised:
+ *         dV = P^T dO,  dP = dO V^T,  dS_ij = P_ij (dP_ij - sum_k P_ik dP_ik),
+ *         dQ = scale dS K,  dK = scale dS^T Q
+ *     (the Jacobian of the row softmax applied to dP, and the chain rule
+ *     through S = scale Q K^T).
  *
  * Every function materialises what the definition materialises (a full score
  * row), loops in the plain order of the formula and uses no blocking, fusion or
@@ -282,5 +289,115 @@ int oracle_attention_prob_row(const double* q, const double* k, const double* v,
                              causal, scale, s, o, &lse, p_out);
     free(s);
     free(o);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Gradients of the definition (one head at a time, every matrix in full).  */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+    const double *q, *k, *v, *dout;
+    double *P, *dS;
+    int64_t N, d;
+    int causal;
+    double scale;
+    int64_t first, stride;
+    double *dq, *dk, *dv;
+} bwd_job_t;
+
+/* Rows: P_i (softmax of the masked, scaled score row), dP_i, dS_i, dQ_i. */
+static void* bwd_rows(void* arg) {
+    bwd_job_t* jb = (bwd_job_t*)arg;
+    const int64_t N = jb->N, d = jb->d;
+    double* dp = (double*)malloc(sizeof(double) * (size_t)N);
+    if (!dp) return NULL;
+    for (int64_t i = jb->first; i < N; i += jb->stride) {
+        double* Pi = jb->P + i * N;
+        double* dSi = jb->dS + i * N;
+        const int64_t n = allowed_keys(i, N, jb->causal);
+        double m = -INFINITY;
+        for (int64_t j = 0; j < n; ++j) {
+            double acc = 0.0;
+            for (int64_t c = 0; c < d; ++c) acc += jb->q[i * d + c] * jb->k[j * d + c];
+            Pi[j] = jb->scale * acc;
+            if (Pi[j] > m) m = Pi[j];
+        }
+        double l = 0.0;
+        for (int64_t j = 0; j < n; ++j) { Pi[j] = exp(Pi[j] - m); l += Pi[j]; }
+        for (int64_t j = 0; j < n; ++j) Pi[j] /= l;
+        for (int64_t j = n; j < N; ++j) Pi[j] = 0.0;
+        /* dP_ij = dO_i . v_j ;  dS_ij = P_ij (dP_ij - sum_k P_ik dP_ik) */
+        double row = 0.0;
+        for (int64_t j = 0; j < n; ++j) {
+            double acc = 0.0;
+            for (int64_t c = 0; c < d; ++c) acc += jb->dout[i * d + c] * jb->v[j * d + c];
+            dp[j] = acc;
+            row += Pi[j] * acc;
+        }
+        for (int64_t j = 0; j < n; ++j) dSi[j] = Pi[j] * (dp[j] - row);
+        for (int64_t j = n; j < N; ++j) dSi[j] = 0.0;
+        /* dQ_i = scale * sum_j dS_ij k_j */
+        for (int64_t c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < n; ++j) acc += dSi[j] * jb->k[j * d + c];
+            jb->dq[i * d + c] = jb->scale * acc;
+        }
+    }
+    free(dp);
+    return NULL;
+}
+
+/* Columns: dV_j = sum_i P_ij dO_i ;  dK_j = scale * sum_i dS_ij q_i. */
+static void* bwd_cols(void* arg) {
+    bwd_job_t* jb = (bwd_job_t*)arg;
+    const int64_t N = jb->N, d = jb->d;
+    for (int64_t j = jb->first; j < N; j += jb->stride) {
+        for (int64_t c = 0; c < d; ++c) {
+            double av = 0.0, ak = 0.0;
+            for (int64_t i = 0; i < N; ++i) {
+                av += jb->P[i * N + j] * jb->dout[i * d + c];
+                ak += jb->dS[i * N + j] * jb->q[i * d + c];
+            }
+            jb->dv[j * d + c] = av;
+            jb->dk[j * d + c] = jb->scale * ak;
+        }
+    }
+    return NULL;
+}
+
+/*
+ * Gradients of L = sum(dO * O) for one head: q, k, v, dout [N, d] fp64 in;
+ * dq, dk, dv [N, d] fp64 out.  Returns 0, -1 on bad arguments, -2 when the
+ * N x N scratch matrices cannot be allocated.
+ */
+int oracle_attention_backward(const double* q, const double* k, const double* v,
+                              const double* dout, int64_t N, int64_t d, int causal, double scale,
+                              double* dq, double* dk, double* dv, int nthreads) {
+    if (!q || !k || !v || !dout || !dq || !dk || !dv || N <= 0 || d <= 0) return -1;
+    double* P = (double*)malloc(sizeof(double) * (size_t)N * (size_t)N);
+    double* dS = (double*)malloc(sizeof(double) * (size_t)N * (size_t)N);
+    if (!P || !dS) { free(P); free(dS); return -2; }
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if ((int64_t)nthreads > N) nthreads = (int)N;
+    bwd_job_t jobs[256];
+    pthread_t th[256];
+    for (int phase = 0; phase < 2; ++phase) {
+        void* (*fn)(void*) = phase == 0 ? bwd_rows : bwd_cols;
+        for (int t = 0; t < nthreads; ++t) {
+            bwd_job_t jb = {q, k, v, dout, P, dS, N, d, causal, scale, t, nthreads, dq, dk, dv};
+            jobs[t] = jb;
+        }
+        int launched = 0;
+        for (int t = 1; t < nthreads; ++t) {
+            if (pthread_create(&th[t], NULL, fn, &jobs[t]) != 0) break;
+            launched = t;
+        }
+        for (int t = launched + 1; t < nthreads; ++t) fn(&jobs[t]);
+        fn(&jobs[0]);
+        for (int t = 1; t <= launched; ++t) pthread_join(th[t], NULL);
+    }
+    free(P);
+    free(dS);
     return 0;
 }

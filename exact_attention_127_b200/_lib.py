@@ -52,6 +52,11 @@ def load_library():
     lib.attn_fwd_host_workspace_bytes.restype = ctypes.c_size_t
     lib.attn_device_status.argtypes = [vp, c_int]
     lib.attn_device_status.restype = c_int
+    lib.attn_bwd_workspace_bytes.argtypes = [i64, i64, i64, i64]
+    lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, c_int,
+                             ctypes.c_float, vp, ctypes.c_size_t, vp]
+    lib.attn_bwd.restype = c_int
     lib.attn_standard_workspace_bytes.argtypes = [i64, i64, i64, i64]
     lib.attn_standard_workspace_bytes.restype = ctypes.c_size_t
     lib.attn_standard.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, c_int, ctypes.c_float,
@@ -187,6 +192,39 @@ def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: boo
             else:
                 torch.cuda.synchronize(device)
     return out, lse
+
+
+def bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(load_library().attn_bwd_workspace_bytes(B, H, N, d))
+
+
+def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+             lse: torch.Tensor, dout: torch.Tensor, causal: bool = False,
+             scale: float | None = None, workspace: torch.Tensor | None = None, stream=None):
+    """Gradients (dq, dk, dv) of the forward pass for upstream gradient dout,
+    recomputed from the saved lse (o, lse from attn_fwd with the same inputs)."""
+    _check_inputs(q, k, v, device_expected=True)
+    for name, t in (("o", o), ("dout", dout)):
+        if t.shape != q.shape or t.dtype != torch.bfloat16 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor shaped like q")
+    B, H, N, d = q.shape
+    if tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    if workspace is None:
+        workspace = torch.empty(max(bwd_workspace_bytes(B, H, N, d), 1), dtype=torch.uint8,
+                                device=q.device)
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        rc = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                          lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
+                          int(bool(causal)), float(scale), workspace.data_ptr(), workspace.numel(),
+                          _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_bwd")
+    return dq, dk, dv
 
 
 def standard_workspace_bytes(B: int, H: int, N: int, d: int) -> int:

@@ -32,7 +32,8 @@ def nvcc_path() -> str:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    deps = SOURCES + [os.path.join(PKG, "csrc", "attn_standard.cuh"), HDR]
+    deps = SOURCES + [os.path.join(PKG, "csrc", f) for f in ("attn_standard.cuh", "attn_bwd.cuh")]
+    deps.append(HDR)
     newest = max(os.path.getmtime(f) for f in deps)
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest:
         return LIB

@@ -44,6 +44,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "attn_fwd.h"
@@ -1067,6 +1068,92 @@ int std_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     return d == 64 ? std_launch<64>(q, k, v, prm, enc, s) : std_launch<128>(q, k, v, prm, enc, s);
 }
 
+#include "attn_bwd.cuh"
+
+/* Backward pass, host side.  Workspace: dQ accumulator (fp32 [BH, N, d]),
+ * D and LSE*log2(e) (fp32 [BH, Np] each), 256-byte aligned pieces. */
+size_t bwd_ws_bytes(int64_t BH, int64_t N, int64_t d) {
+    const int64_t Np = (N + BLOCK_M - 1) / BLOCK_M * BLOCK_M;
+    auto a256 = [](size_t x) { return (x + 255u) & ~static_cast<size_t>(255u); };
+    return a256(static_cast<size_t>(BH) * N * d * 4) + 2 * a256(static_cast<size_t>(BH) * Np * 4);
+}
+
+template <int D, bool CAUSAL>
+int bwd_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+               const CUtensorMap& mdo, const __nv_bfloat16* o, const __nv_bfloat16* dout,
+               const float* lse, const BwdParams& prm, cudaStream_t stream) {
+    auto kern = bwd_main_kernel<D, CAUSAL>;
+    constexpr int SMEM = BwdCfg<D>::SMEM_BYTES;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_LAUNCH;
+    }
+    const int64_t prows = static_cast<int64_t>(prm.BH) * prm.Np;
+    bwd_pre_kernel<D><<<static_cast<unsigned>((prows + 7) / 8), 256, 0, stream>>>(
+        o, dout, lse, const_cast<float*>(prm.Dp), const_cast<float*>(prm.lse2), prm.dq_acc, prm.N,
+        prm.Np, prm.BH);
+    kern<<<dim3(prm.nblk, prm.BH), BWD_THREADS, SMEM, stream>>>(mq, mk, mv, mdo, prm);
+    const int64_t n = static_cast<int64_t>(prm.BH) * prm.N * D;
+    bwd_post_kernel<<<static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 148 * 16)), 256, 0,
+                      stream>>>(prm.dq_acc, prm.dq, n);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+    return ATTN_OK;
+}
+
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N,
+             int64_t d, int causal, float scale, void* workspace, size_t workspace_bytes,
+             void* stream) {
+    bool empty = false;
+    int st = validate_shape(B, H, N, d, scale, &empty);
+    if (st != ATTN_OK || empty) return st;
+    if (B * H > 65535) return ATTN_ERR_SHAPE;
+    const void* ptrs[9] = {q, k, v, o, dout, lse, dq, dk, dv};
+    for (const void* ptr : ptrs) {
+        if (!ptr) return ATTN_ERR_NULL;
+        if (reinterpret_cast<uintptr_t>(ptr) & 15u) return ATTN_ERR_ALIGN;
+    }
+    const int64_t BH = B * H;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+        workspace_bytes < bwd_ws_bytes(BH, N, d))
+        return ATTN_ERR_WORKSPACE;
+    int dev = 0;
+    DeviceInfo* di = nullptr;
+    if ((st = device_info(&dev, &di)) != ATTN_OK) return st;
+    EncodeTiledFn enc = nullptr;
+    if ((st = get_encode(&enc)) != ATTN_OK) return st;
+    CUtensorMap mq, mk, mv, mdo;
+    if ((st = encode_map(enc, &mq, q, BH, N, d)) != ATTN_OK) return st;
+    if ((st = encode_map(enc, &mk, k, BH, N, d)) != ATTN_OK) return st;
+    if ((st = encode_map(enc, &mv, v, BH, N, d)) != ATTN_OK) return st;
+    if ((st = encode_map(enc, &mdo, dout, BH, N, d)) != ATTN_OK) return st;
+    const int64_t Np = (N + BLOCK_M - 1) / BLOCK_M * BLOCK_M;
+    auto a256 = [](size_t x) { return (x + 255u) & ~static_cast<size_t>(255u); };
+    char* ws = static_cast<char*>(workspace);
+    BwdParams prm;
+    prm.dq = static_cast<__nv_bfloat16*>(dq);
+    prm.dk = static_cast<__nv_bfloat16*>(dk);
+    prm.dv = static_cast<__nv_bfloat16*>(dv);
+    prm.dq_acc = reinterpret_cast<float*>(ws);
+    prm.Dp = reinterpret_cast<float*>(ws + a256(static_cast<size_t>(BH) * N * d * 4));
+    prm.lse2 = prm.Dp + (a256(static_cast<size_t>(BH) * Np * 4) / 4);
+    prm.N = static_cast<int>(N);
+    prm.Np = static_cast<int>(Np);
+    prm.BH = static_cast<int>(BH);
+    prm.nblk = static_cast<int>(Np / BLOCK_M);
+    prm.scale = scale;
+    prm.scale_log2 = scale * LOG2E;
+    prm.wait_limit_ns = WAIT_LIMIT_NS;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const auto* ob = static_cast<const __nv_bfloat16*>(o);
+    const auto* db = static_cast<const __nv_bfloat16*>(dout);
+    if (d == 64)
+        return causal ? bwd_launch<64, true>(mq, mk, mv, mdo, ob, db, lse, prm, s)
+                      : bwd_launch<64, false>(mq, mk, mv, mdo, ob, db, lse, prm, s);
+    return causal ? bwd_launch<128, true>(mq, mk, mv, mdo, ob, db, lse, prm, s)
+                  : bwd_launch<128, false>(mq, mk, mv, mdo, ob, db, lse, prm, s);
+}
+
 /* The forward call behind attn_fwd and the timeout test hook. */
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
              int64_t H, int64_t N, int64_t d, int causal, float scale, void* stream,
@@ -1126,6 +1213,20 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
 int attn_fwd_test_wait_timeout(const void* q, const void* k, const void* v, void* o, float* lse,
                                int64_t B, int64_t H, int64_t N, int64_t d, void* stream) {
     return fwd_impl(q, k, v, o, lse, B, H, N, d, 0, 0.125f, stream, TEST_WAIT_LIMIT_NS, 1);
+}
+
+size_t attn_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {
+    bool empty = false;
+    if (validate_shape(B, H, N, d, 1.0f, &empty) != ATTN_OK || empty || B * H > 65535) return 0;
+    return bwd_ws_bytes(B * H, N, d);
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N,
+             int64_t d, int causal, float scale, void* workspace, size_t workspace_bytes,
+             void* stream) {
+    return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, workspace,
+                    workspace_bytes, stream);
 }
 
 size_t attn_standard_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {

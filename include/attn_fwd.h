@@ -102,6 +102,35 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
 int attn_device_status(void* stream, int reset);
 
 /*
+ * attn_bwd_workspace_bytes -- device workspace attn_bwd needs: an fp32 dQ
+ * accumulator [B, H, N, d] plus two fp32 [B, H, Np] vectors (Np = N rounded
+ * up to 128), 256-byte aligned pieces.  0 for invalid or empty shapes.
+ */
+size_t attn_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
+
+/*
+ * attn_bwd -- gradients of the forward pass with respect to q, k and v, by
+ * recomputation from the saved LSE ("science-depth-m4-047", section 3, point
+ * (c)): no N x N matrix reaches device memory.  With s_ij = scale q_i . k_j and
+ * P_ij = exp(s_ij - LSE_i) (masked j > i when causal):
+ *     dV = P^T dO,  dS = P * (dO V^T - D),  D_i = sum_c dO_ic O_ic,
+ *     dQ = scale dS K,  dK = scale dS^T Q.
+ *   q, k, v, o, dout : device, bf16 [B, H, N, d] (o and lse from attn_fwd with
+ *                      the same q, k, v, causal, scale), read only.
+ *   lse              : device, fp32 [B, H, N], read only.
+ *   dq, dk, dv       : device, bf16 [B, H, N, d], written.
+ *   workspace        : device, >= attn_bwd_workspace_bytes, 256-byte aligned,
+ *                      caller-owned, contents ignored on entry; calls that
+ *                      overlap on the GPU must not share it.
+ * Three kernels are enqueued on `stream`.  Same d, scale, alignment and error
+ * conventions as attn_fwd; additionally B*H <= 65535.
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N,
+             int64_t d, int causal, float scale, void* workspace, size_t workspace_bytes,
+             void* stream);
+
+/*
  * attn_standard_workspace_bytes -- device workspace attn_standard needs: the
  * N x N score matrix of every head in fp32, rows padded to a multiple of 128
  * (4 * B * H * Np^2 bytes, Np = N rounded up to 128).  0 for invalid shapes.

@@ -1,0 +1,94 @@
+"""Backward pass: dq, dk, dv from the CUDA path (recomputed from the saved LSE)
+against the fp64 gradients of the textbook definition.
+
+Tolerance (derived from the arithmetic): P and dS enter the tensor cores as
+bf16 (relative rounding 2^-9 per element) and the outputs are rounded to bf16
+once (2^-9); accumulations are fp32.  Per tensor we require relative L2 error
+<= 1e-2 and max |error| <= 3e-2 * max |reference| + 1e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_127_b200 as attn
+import oracle
+from exact_attention_127_b200 import inputs
+
+REL_L2 = 1e-2
+MAX_REL = 3e-2
+FAKE = 0x10000
+
+
+def test_backward_validation_on_host():
+    lib = attn.load_library()
+    a = [FAKE + 0x100000 * i for i in range(9)]
+    big = 1 << 40
+    assert lib.attn_bwd(*a, 1, 1, 100, 96, 0, 0.1, FAKE + 0x1000000, big, None) == -3
+    assert lib.attn_bwd(*a, 1, 70000, 100, 64, 0, 0.1, FAKE + 0x1000000, big, None) == -4
+    assert lib.attn_bwd(*a, 1, 1, 100, 64, 0, 0.1, None, big, None) == -11
+    a2 = list(a)
+    a2[5] = None
+    assert lib.attn_bwd(*a2, 1, 1, 100, 64, 0, 0.1, FAKE + 0x1000000, big, None) == -1
+    need = lib.attn_bwd_workspace_bytes(2, 3, 100, 64)
+    assert need >= 2 * 3 * 100 * 64 * 4 + 2 * 2 * 3 * 128 * 4
+
+
+def _grads(q, k, v, dout, causal, scale):
+    qd, kd, vd, dd = (t.cuda() for t in (q, k, v, dout))
+    o, lse = attn.attn_fwd(qd, kd, vd, causal=causal, scale=scale)
+    dq, dk, dv = attn.attn_bwd(qd, kd, vd, o, lse, dd, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert attn.device_status(reset=True) == 0
+    return dq.cpu(), dk.cpu(), dv.cpu()
+
+
+def _check(q, k, v, dout, causal, scale, label):
+    B, H, N, d = q.shape
+    got = _grads(q, k, v, dout, causal, scale)
+    ref = oracle.attention_backward(q, k, v, dout, causal, scale)
+    for name, g, r in zip(("dq", "dk", "dv"), got, ref):
+        gf = g.reshape(B * H, N, d).double().numpy()
+        err = np.abs(gf - r)
+        rel = np.linalg.norm(gf - r) / max(np.linalg.norm(r), 1e-30)
+        msg = f"{label} {name}: relL2={rel:.3e} max|err|={err.max():.3e} max|ref|={np.abs(r).max():.3e}"
+        print(msg)
+        assert np.all(np.isfinite(gf)), msg
+        if np.linalg.norm(r) > 1e-6:          # an all-zero reference has no relative error
+            assert rel <= REL_L2, msg
+        assert err.max() <= MAX_REL * np.abs(r).max() + 1e-3, msg
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 100, 128, 129, 300, 700])
+def test_backward_matches_oracle(N, d, causal):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    q, k, v = inputs.make_qkv(1, 2, N, d, seed=400 + N)
+    dout = inputs.make_qkv(1, 2, N, d, seed=500 + N)[0]
+    _check(q, k, v, dout, causal, 1 / math.sqrt(d), f"N={N} d={d} causal={causal}")
+
+
+@pytest.mark.gpu
+def test_backward_larger_causal_two_heads():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    q, k, v = inputs.make_qkv(1, 2, 2048, 128, seed=41)
+    dout = inputs.make_qkv(1, 2, 2048, 128, seed=42)[0]
+    _check(q, k, v, dout, True, 1 / math.sqrt(128), "N=2048 d=128 causal")
+
+
+@pytest.mark.gpu
+def test_backward_deterministic_dk_dv():
+    """dK and dV are written once per K/V block (no atomics): bit-identical reruns."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    q, k, v = inputs.make_qkv(2, 2, 1000, 64, seed=43)
+    dout = inputs.make_qkv(2, 2, 1000, 64, seed=44)[0]
+    a = _grads(q, k, v, dout, True, 0.125)
+    b = _grads(q, k, v, dout, True, 0.125)
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    assert (a[0].float() - b[0].float()).abs().max().item() <= 1e-2   # dQ uses fp32 atomics

@@ -402,6 +402,63 @@ def run_cuda(args, w):
 DECODE_METRIC = "split-K/V decode attention GB/s (K/V cache bytes read / time)"
 
 
+BWD_METRIC = "attention bwd TFLOP/s (2.5 x forward FLOPs: five GEMMs)"
+
+
+def run_backward(args, w):
+    """One step = one attn_bwd call (D/LSE preparation, the fused backward
+    kernel, dQ conversion) on a forward workload; tensor-core bound."""
+    import torch
+
+    import exact_attention_127_b200 as attn
+
+    rank, local, world = dist_env()
+    if world > 1:
+        raise SystemExit("--pass bwd runs on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    attn.load_library()
+    q, k, v = (t.to(dev) for t in _inputs.workload_inputs(w))
+    dout = _inputs.make_qkv(w.B, w.H, w.N, w.d, w.seed + 100)[0].to(dev)
+    o, lse = attn.attn_fwd(q, k, v, causal=w.causal, scale=w.scale)
+    ws = torch.empty(attn.bwd_workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            attn.attn_bwd(q, k, v, o, lse, dout, w.causal, w.scale, workspace=ws, stream=stream)
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    sampler.start()
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            attn.attn_bwd(q, k, v, o, lse, dout, w.causal, w.scale, workspace=ws, stream=stream)
+    e1.record(stream)
+    stream.synchronize()
+    sampler.stop()
+    if attn.device_status(reset=True, stream=stream) != 0:
+        raise RuntimeError("device-side error in the backward pass")
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = 2.5 * w.flops()
+    peaks, peak_src = load_peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+    line = {
+        "metric": BWD_METRIC, "value": tf, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(w, 1),
+        "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"], "traffic": None,
+                     "peak_source": f"{peak_src} bf16 dense matmul, burst (MEASURED_PEAKS.json)",
+                     "kernel": "bwd_pre_kernel + bwd_main_kernel + bwd_post_kernel",
+                     "algorithmic_flops_per_launch": flops},
+        "e2e": None, "gpu_launches": 3 * args.steps, "clocks": sampler.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_standard(args, w):
     """The unfused three-kernel path on a forward workload (context for the
     fused kernel): same metric (useful TFLOP/s); its roofline is HBM, since the
@@ -567,6 +624,8 @@ def main(argv=None):
     ap.add_argument("--ref-step-seconds", type=float, default=2.0)
     ap.add_argument("--ref-budget-seconds", type=float, default=150.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
+                    help="forward (default) or the backward pass of the workload")
     ap.add_argument("--path", default="fused", choices=["fused", "standard"],
                     help="fused kernel (default) or the unfused three-kernel path for comparison")
     ap.add_argument("--batch", type=int, default=None,
@@ -591,6 +650,8 @@ def main(argv=None):
         sys.stderr.write(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE\n")
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.pass_ == "bwd":
+        return run_backward(args, w)
     if args.path == "standard":
         return run_standard(args, w)
     return run_cuda(args, w)

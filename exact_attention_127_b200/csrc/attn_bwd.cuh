@@ -12,24 +12,34 @@
  *     dQ_i  = scale sum_j dS_ij k_j,   dK_j = scale sum_i dS_ij q_i
  * No N x N matrix reaches device memory.
  *
- * bwd_pre_kernel   D_i and LSE_i * log2(e) into row-padded workspace arrays; zero
- *                  the fp32 dQ accumulator.
+ * bwd_pre_kernel   D_i and LSE_i * log2(e) into row-padded workspace arrays (the
+ *                  host zeroes the fp32 dQ accumulator before it).
  * bwd_main_kernel  one CTA per (head, 128-row K/V block j), looping over the Q
  *                  blocks i that see block j.  K_j and V_j stay in shared memory;
  *                  Q_i and dO_i stream through a 2-stage TMA ring.  Per i, on
  *                  the tensor cores (TMEM accumulators):
  *                      S^T  = K_j Q_i^T   -> TMEM A      dP^T = V_j dO_i^T -> TMEM B
- *                  warps 0-3 (thread = K/V row = TMEM lane) turn them into P^T
- *                  (bf16, over TMEM A) and scale * dS^T (bf16, over TMEM B, and
- *                  into shared memory as dS), then
- *                      dV_j += P^T dO_i  (A from TMEM)    dK_j += dS^T Q_i  (A from TMEM)
- *                      dQ_i partial = dS K_j  (A, B from shared memory) -> TMEM A
- *                  and warps 4-7 add the dQ partial into the fp32 accumulator
- *                  with vector atomics.  At the end warps 4-7 write dK_j, dV_j.
+ *                  warps 0-7 (thread = K/V row = TMEM lane; warps w and w+4 share
+ *                  the lanes and split the 128 queries in halves) turn S^T into
+ *                  P^T (bf16, packed over the first half of its own columns of
+ *                  TMEM A) and, once dP^T is there, scale * dS (bf16) into shared
+ *                  memory; then
+ *                      dQ_i partial = dS K_j          (A, B from shared memory) -> TMEM dQ
+ *                      dV_j += P^T dO_i               (A from TMEM)
+ *                      S^T of block i+1               (overwrites P^T: MMAs run in issue order)
+ *                      dK_j += dS^T Q_i               (A, B from shared memory)
+ *                  and the same 8 warps add the dQ partial into the fp32
+ *                  accumulator with vector atomics while the tensor cores
+ *                  already work on block i+1.  At the end they write dK_j, dV_j.
  * bwd_post_kernel  dQ accumulator -> bf16.
+ *
+ * The dQ accumulator is tiled [BH][Q block][D/4][128 rows][4]: the four
+ * columns a thread adds with one vector atomic sit next to those of the rows
+ * beside it, so a warp's atomic covers 512 contiguous bytes.
  */
 
-constexpr int BWD_THREADS = 320;    // warps 0-3 dS, 4-7 dQ readout + epilogue, 8 TMA, 9 MMA
+constexpr int BWD_THREADS = 320;    // warps 0-7 P, dS, dQ readout, epilogue; 8 TMA; 9 MMA
+constexpr int BWD_COMPUTE = 256;
 constexpr int BWD_LOAD_WARP = 8;
 constexpr int BWD_MMA_WARP = 9;
 
@@ -37,7 +47,7 @@ struct BwdParams {
     __nv_bfloat16* dq;
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
-    float* dq_acc;       // [BH, N, D] fp32
+    float* dq_acc;       // [BH, Np/128, D/4, 128, 4] fp32
     const float* Dp;     // [BH, Np]  D_i, zero-padded
     const float* lse2;   // [BH, Np]  LSE_i * log2(e), zero-padded
     int N, Np, BH, nblk;
@@ -55,10 +65,14 @@ struct BwdCfg {
     static constexpr uint32_t DO_OFF = 4 * TILE;                // [2] stages
     static constexpr uint32_t DS_OFF = 6 * TILE;                // 128 x 128 bf16 = 32 KB
     static constexpr uint32_t BAR_OFF = DS_OFF + 32768;
-    static constexpr int NUM_BARS = 1 + 4 + 6;
+    static constexpr int NUM_BARS = 12;
     static constexpr uint32_t MISC_OFF = BAR_OFF + 8 * NUM_BARS;
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+    // TMEM columns: S^T / P^T, dP^T, the dV and dK accumulators, the dQ partial
+    // (over dP^T when no columns are left, i.e. at D = 128)
     static constexpr uint32_t RA = 0, RB = 128, DV_COL = 256, DK_COL = 256 + D;
+    static constexpr uint32_t DQ_COL = (256 + 2 * D + D <= 512) ? 256 + 2 * D : RB;
+    static constexpr bool DQ_OVER_DP = DQ_COL == RB;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
@@ -68,13 +82,18 @@ __host__ __device__ constexpr uint32_t idesc_bf16_ab(int M, int N, bool a_mn, bo
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-/* D_i = dO_i . O_i, lse2_i = LSE_i log2(e) (zero past N), dq_acc = 0.
- * One warp per padded row. */
+/* TMEM column of the packed P^T columns for queries [16 kk, 16 kk + 16): the
+ * half h = kk / 4 of the queries is packed at the start of its own 64 columns. */
+__device__ __forceinline__ uint32_t bwd_p_col(int kk) {
+    return static_cast<uint32_t>((kk >> 2) * 64 + (kk & 3) * 8);
+}
+
+/* D_i = dO_i . O_i, lse2_i = LSE_i log2(e) (zero past N).  One warp per padded row. */
 template <int D>
 __global__ void __launch_bounds__(256)
 bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                const float* __restrict__ lse, float* __restrict__ Dp, float* __restrict__ lse2,
-               float* __restrict__ dq_acc, int N, int Np, int BH) {
+               int N, int Np, int BH) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t prow = static_cast<int64_t>(blockIdx.x) * 8 + warp;     // over BH * Np
     if (prow >= static_cast<int64_t>(BH) * Np) return;
@@ -83,10 +102,8 @@ bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restr
     if (i < N) {
         const int64_t base = (static_cast<int64_t>(bh) * N + i) * D;
 #pragma unroll
-        for (int c = lane; c < D; c += 32) {
+        for (int c = lane; c < D; c += 32)
             dsum += __bfloat162float(o[base + c]) * __bfloat162float(dout[base + c]);
-            dq_acc[base + c] = 0.0f;
-        }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
@@ -96,11 +113,31 @@ bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restr
     }
 }
 
-__global__ void bwd_post_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
-                                int64_t n) {
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-        dq[i] = __float2bfloat16_rn(acc[i]);
+/* Tiled fp32 dQ accumulator -> bf16 [BH, N, D].  One CTA per (head, Q block):
+ * coalesced reads of the tile, a transpose through shared memory, and a
+ * contiguous copy of the block's rows. */
+template <int D>
+__global__ void __launch_bounds__(BLOCK_M)
+bwd_post_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, int N, int nblk) {
+    constexpr int ROW = D + 8;                   // padded bf16 row: fewer bank conflicts
+    __shared__ __align__(16) __nv_bfloat16 tile[BLOCK_M * ROW];
+    const int t = threadIdx.x;
+    const int bh = blockIdx.x / nblk, ib = blockIdx.x % nblk;
+    const float4* src = reinterpret_cast<const float4*>(acc) +
+                        static_cast<int64_t>(blockIdx.x) * (D / 4) * BLOCK_M;
+#pragma unroll 4
+    for (int g = 0; g < D / 4; ++g) {
+        const float4 v = src[g * BLOCK_M + t];
+        *reinterpret_cast<uint2*>(&tile[t * ROW + 4 * g]) =
+            make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+    }
+    __syncthreads();
+    const int rows = min(BLOCK_M, N - ib * BLOCK_M);
+    uint4* dst = reinterpret_cast<uint4*>(dq + (static_cast<int64_t>(bh) * N + ib * BLOCK_M) * D);
+    for (int i = t; i < rows * (D / 8); i += BLOCK_M) {
+        const int row = i / (D / 8), c16 = i % (D / 8);
+        dst[i] = *reinterpret_cast<const uint4*>(&tile[row * ROW + c16 * 8]);
+    }
 }
 
 template <int D, bool CAUSAL>
@@ -120,7 +157,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     auto bar_full = [&](int s) { return bars + 8 + 8u * s; };
     auto bar_empty = [&](int s) { return bars + 24 + 8u * s; };
     const uint32_t bar_s = bars + 40, bar_p = bars + 48, bar_dq = bars + 56, bar_dqf = bars + 64;
-    const uint32_t bar_dkv = bars + 72, bar_drain = bars + 80;
+    const uint32_t bar_dkv = bars + 72, bar_drain = bars + 80, bar_dp = bars + 88;
     uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::MISC_OFF);
     volatile uint32_t* const abort_flag = reinterpret_cast<volatile uint32_t*>(base_ptr + C::MISC_OFF + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -136,9 +173,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(bar_empty(s), 1);
         }
         mbar_init(bar_s, 1);
-        mbar_init(bar_p, BLOCK_M);
+        mbar_init(bar_dp, 1);
+        mbar_init(bar_p, BWD_COMPUTE);
         mbar_init(bar_dq, 1);
-        mbar_init(bar_dqf, BLOCK_M);
+        mbar_init(bar_dqf, BWD_COMPUTE);
         mbar_init(bar_dkv, 1);
         mbar_init(bar_drain, 1);
         *abort_flag = 0u;
@@ -193,44 +231,67 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             constexpr uint32_t ID_ACC = idesc_bf16_ab(BLOCK_M, D, false, true);        // dV, dK
             constexpr uint32_t ID_DQ = idesc_bf16_ab(BLOCK_M, D, true, true);          // dQ
             const uint32_t ta = tmem + C::RA, tb = tmem + C::RB;
-            const uint32_t tdv = tmem + C::DV_COL, tdk = tmem + C::DK_COL;
+            const uint32_t tdv = tmem + C::DV_COL, tdk = tmem + C::DK_COL, tdq = tmem + C::DQ_COL;
             const uint64_t kd = sdesc_sw128(sK, 16, 1024);                  // K-major
             const uint64_t vd = sdesc_sw128(sV, 16, 1024);                  // K-major
             const uint64_t k_mn = sdesc_sw128(sK, CHUNK_BYTES, 1024);       // K_j as MN-major B
-            const uint64_t ds_mn = sdesc_sw128(sDS, 16384, 1024);           // dS as MN-major A
+            const uint64_t ds_mn = sdesc_sw128(sDS, 16384, 1024);           // dS as MN-major A (dQ)
+            const uint64_t ds_k = sdesc_sw128(sDS, 16, 1024);               // dS^T as K-major A (dK)
             bool ok = mbar_wait(bar_kv, 0, abort_flag, wlim);
+            if (ok) ok = mbar_wait(bar_full(0), 0, abort_flag, wlim);
+            if (ok) {
+                tc_fence_after();
+                issue_qk<D>(ta, kd, sdesc_sw128(base + C::Q_OFF, 16, 1024), ID_KQ);  // S^T = K Q^T
+                mma_commit(bar_s);
+            }
             for (int it = 0; it < nq && ok; ++it) {
                 const int s = it & 1;
-                ok = mbar_wait(bar_full(s), (it >> 1) & 1, abort_flag, wlim);
-                if (!ok) break;
-                if (it > 0) {
-                    // the dQ partial of the previous block has been read out of TMEM A
+                const uint32_t sq = base + C::Q_OFF + s * TILE, sdo = base + C::DO_OFF + s * TILE;
+                if (C::DQ_OVER_DP && it > 0) {
+                    // dP^T overwrites the previous dQ partial: wait until it was read out
                     ok = mbar_wait(bar_dqf, (it - 1) & 1, abort_flag, wlim);
                     if (!ok) break;
                     tc_fence_after();
                 }
-                const uint32_t sq = base + C::Q_OFF + s * TILE, sdo = base + C::DO_OFF + s * TILE;
-                issue_qk<D>(ta, kd, sdesc_sw128(sq, 16, 1024), ID_KQ);          // S^T = K Q^T
                 issue_qk<D>(tb, vd, sdesc_sw128(sdo, 16, 1024), ID_KQ);         // dP^T = V dO^T
-                mma_commit(bar_s);
+                mma_commit(bar_dp);
                 ok = mbar_wait(bar_p, it & 1, abort_flag, wlim);
                 if (!ok) break;
                 tc_fence_after();
+                if (!C::DQ_OVER_DP && it > 0) {
+                    ok = mbar_wait(bar_dqf, (it - 1) & 1, abort_flag, wlim);
+                    if (!ok) break;
+                    tc_fence_after();
+                }
                 const uint64_t do_mn = sdesc_sw128(sdo, CHUNK_BYTES, 1024);
                 const uint64_t q_mn = sdesc_sw128(sq, CHUNK_BYTES, 1024);
 #pragma unroll
                 for (int kk = 0; kk < BLOCK_M / 16; ++kk) {
                     const uint64_t off = static_cast<uint64_t>((kk * 16 * 128) >> 4);
-                    const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                    mma_ts(tdv, ta + kk * 8, do_mn + off, ID_ACC, acc);         // dV += P^T dO
-                    mma_ts(tdk, tb + kk * 8, q_mn + off, ID_ACC, acc);          // dK += dS^T Q
+                    mma_ss(tdq, ds_mn + off, k_mn + off, ID_DQ, kk > 0 ? 1u : 0u);  // dQ = dS K
                 }
+                mma_commit(bar_dq);
 #pragma unroll
                 for (int kk = 0; kk < BLOCK_M / 16; ++kk) {
                     const uint64_t off = static_cast<uint64_t>((kk * 16 * 128) >> 4);
-                    mma_ss(ta, ds_mn + off, k_mn + off, ID_DQ, kk > 0 ? 1u : 0u);  // dQ = dS K
+                    mma_ts(tdv, ta + bwd_p_col(kk), do_mn + off, ID_ACC,
+                           (it > 0 || kk > 0) ? 1u : 0u);                         // dV += P^T dO
                 }
-                mma_commit(bar_dq);
+                if (it + 1 < nq) {
+                    const int s1 = s ^ 1;
+                    ok = mbar_wait(bar_full(s1), ((it + 1) >> 1) & 1, abort_flag, wlim);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_qk<D>(ta, kd, sdesc_sw128(base + C::Q_OFF + s1 * TILE, 16, 1024), ID_KQ);
+                    mma_commit(bar_s);
+                }
+#pragma unroll
+                for (int kk = 0; kk < BLOCK_M / 16; ++kk) {
+                    const uint64_t off_mn = static_cast<uint64_t>((kk * 16 * 128) >> 4);
+                    const uint64_t off_k = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+                    mma_ss(tdk, ds_k + off_k, q_mn + off_mn, ID_ACC,
+                           (it > 0 || kk > 0) ? 1u : 0u);                         // dK += dS^T Q
+                }
                 mma_commit(bar_empty(s));
             }
             if (ok) mma_commit(bar_dkv);
@@ -238,94 +299,103 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_drain_wait(bar_drain, 0, wlim);
         }
         __syncwarp();
-    } else if (warp < 4) {
-        /* ---------------- P^T and dS^T, thread = K/V row (TMEM lane) ---------------- */
-        const int r = warp * 32 + lane;
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    } else {
+        /* ---------------- warps 0-7: P^T, dS, dQ readout, dK/dV epilogue ----------------
+         * thread = TMEM lane: K/V row r while P and dS are formed, query row r
+         * while dQ is read out; warp w covers lanes 32 (w % 4) .. and the half
+         * h = w / 4 of the columns. */
+        const int quarter = warp & 3, h = warp >> 2;
+        const int r = quarter * 32 + lane;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
         const float c = p.scale_log2, sc = p.scale;
-        const int kv = jb * BLOCK_M + r;
+        bool ok = true;
         for (int it = 0; it < nq; ++it) {
             const int ib = ib0 + it;
-            bool ok = mbar_wait(bar_s, it & 1, abort_flag, wlim);
+            ok = mbar_wait(bar_s, it & 1, abort_flag, wlim);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            const float* lse2 = p.lse2 + static_cast<int64_t>(bh) * p.Np + ib * BLOCK_M;
-            const float* dvec = p.Dp + static_cast<int64_t>(bh) * p.Np + ib * BLOCK_M;
-            const bool diag = CAUSAL && ib == jb;
-#pragma unroll 1
-            for (int ch = 0; ch < BLOCK_M / 32; ++ch) {
-                uint32_t sv[32], dpv[32];
-                tmem_ld32_wait(lane_base + C::RA + ch * 32, sv);
-                tmem_ld32_wait(lane_base + C::RB + ch * 32, dpv);
-                uint32_t pk[16], dk[16];
+            const int64_t row0 = static_cast<int64_t>(bh) * p.Np + ib * BLOCK_M + 64 * h;
+            const float* lse2 = p.lse2 + row0;
+            const float* dvec = p.Dp + row0;
+            // on the diagonal block key r is masked for the queries before it:
+            // column ch * 32 + e of this half is masked when it is < mask_lim
+            const int mask_lim = (CAUSAL && ib == jb) ? r - 64 * h : 0;
+            float pf[64];
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                uint32_t sv[32];
+                tmem_ld32_wait(lane_base + C::RA + 64 * h + 32 * ch, sv);
+                uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {
                     const float4 l4 = __ldg(reinterpret_cast<const float4*>(lse2 + ch * 32 + e));
-                    const float4 d4 = __ldg(reinterpret_cast<const float4*>(dvec + ch * 32 + e));
                     const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                    const float dvv[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float pp[4], dd[4];
 #pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const int ql = ch * 32 + e + h;
-                        float pv = ex2(fmaf(__uint_as_float(sv[e + h]), c, -lv[h]));
-                        if (diag && ql < r) pv = 0.0f;        // key kv row r masked for query ql < r
-                        pp[h] = pv;
-                        dd[h] = pv * (__uint_as_float(dpv[e + h]) - dvv[h]) * sc;
+                    for (int hh = 0; hh < 4; ++hh) {
+                        float pv = ex2(fmaf(__uint_as_float(sv[e + hh]), c, -lv[hh]));
+                        if (ch * 32 + e + hh < mask_lim) pv = 0.0f;
+                        pf[ch * 32 + e + hh] = pv;
                     }
-                    pk[e / 2] = pack_bf16(pp[0], pp[1]);
-                    pk[e / 2 + 1] = pack_bf16(pp[2], pp[3]);
+                    pk[e / 2] = pack_bf16(pf[ch * 32 + e], pf[ch * 32 + e + 1]);
+                    pk[e / 2 + 1] = pack_bf16(pf[ch * 32 + e + 2], pf[ch * 32 + e + 3]);
+                }
+                tmem_st16(lane_base + C::RA + 64 * h + 16 * ch, pk);
+            }
+            ok = mbar_wait(bar_dp, it & 1, abort_flag, wlim);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            // dS into shared memory: 64-query atoms 16 KB apart, K/V row r at 128 B,
+            // 8-row groups 1 KB apart, 16-byte units swizzled by r % 8 -- the MN-major
+            // A operand of dQ = dS K and the K-major A operand of dK = dS^T Q
+            const uint32_t atom = sDS + h * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                uint32_t dpv[32];
+                tmem_ld32_wait(lane_base + C::RB + 64 * h + 32 * ch, dpv);
+                uint32_t dk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) {
+                    const float4 d4 = __ldg(reinterpret_cast<const float4*>(dvec + ch * 32 + e));
+                    const float dvv[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float dd[4];
+#pragma unroll
+                    for (int hh = 0; hh < 4; ++hh)
+                        dd[hh] = pf[ch * 32 + e + hh] * (__uint_as_float(dpv[e + hh]) - dvv[hh]) * sc;
                     dk[e / 2] = pack_bf16(dd[0], dd[1]);
                     dk[e / 2 + 1] = pack_bf16(dd[2], dd[3]);
                 }
-                tmem_st16(lane_base + C::RA + ch * 16, pk);
-                tmem_st16(lane_base + C::RB + ch * 16, dk);
-                // dS into shared memory as the MN-major A operand of dQ = dS K:
-                // query index contiguous in 64-wide atoms (16 KB apart), K/V row r
-                // at 128 B, 8-row groups 1 KB apart, 16-byte units swizzled by r % 8
-                const uint32_t atom = sDS + (ch >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int unit = (ch & 1) * 4 + u;
+                    const int unit = ch * 4 + u;
                     const uint32_t addr = atom + ((unit ^ (r & 7)) << 4);
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
                                  "r"(dk[4 * u]), "r"(dk[4 * u + 1]), "r"(dk[4 * u + 2]),
                                  "r"(dk[4 * u + 3]) : "memory");
                 }
             }
-            (void)kv;
             tmem_wait_st();
             tc_fence_before();
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // dS visible to the MMA
             mbar_arrive(bar_p);
-        }
-    } else if (warp < 8) {
-        /* ---------------- dQ readout (thread = query row) and the dK, dV epilogue ---------------- */
-        const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-        bool ok = true;
-        for (int it = 0; it < nq; ++it) {
-            const int ib = ib0 + it;
+
+            // dQ partial (thread = query row r) into the tiled accumulator
             ok = mbar_wait(bar_dq, it & 1, abort_flag, wlim);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            const int row = ib * BLOCK_M + r;
-            float* dst = p.dq_acc + (static_cast<int64_t>(bh) * p.N + (row < p.N ? row : 0)) * D;
+            float* dst = p.dq_acc + (static_cast<int64_t>(bh) * p.nblk + ib) * (BLOCK_M * D) + r * 4;
 #pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
+            for (int ch = 0; ch < D / 64; ++ch) {
+                const int c0 = h * (D / 2) + ch * 32;
                 uint32_t v[32];
-                tmem_ld32_wait(lane_base + C::RA + ch * 32, v);
-                if (row < p.N) {
+                tmem_ld32_wait(lane_base + C::DQ_COL + c0, v);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        atomicAdd(reinterpret_cast<float4*>(dst + ch * 32 + 4 * e),
-                                  make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                              __uint_as_float(v[4 * e + 2]),
-                                              __uint_as_float(v[4 * e + 3])));
-                }
+                for (int e = 0; e < 8; ++e)
+                    atomicAdd(reinterpret_cast<float4*>(dst + (c0 / 4 + e) * (BLOCK_M * 4)),
+                              make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                          __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])));
             }
             tc_fence_before();
             mbar_arrive(bar_dqf);
@@ -335,27 +405,25 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             ok = __all_sync(0xffffffffu, ok);
         }
         if (ok) {
+            // warps 0-3 write dV_j, warps 4-7 dK_j (thread = K/V row r)
             tc_fence_after();
             const int kvrow = jb * BLOCK_M + r;
             const int64_t off = (static_cast<int64_t>(bh) * p.N + (kvrow < p.N ? kvrow : 0)) * D;
+            __nv_bfloat16* out = (h ? p.dk : p.dv) + off;
+            const uint32_t col = h ? C::DK_COL : C::DV_COL;
 #pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                __nv_bfloat16* out = (which ? p.dk : p.dv) + off;
-                const uint32_t col = which ? C::DK_COL : C::DV_COL;
+            for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t v[32];
+                tmem_ld32_wait(lane_base + col + ch * 32, v);
+                if (kvrow < p.N) {
+                    uint4* d4 = reinterpret_cast<uint4*>(out + ch * 32);
 #pragma unroll
-                for (int ch = 0; ch < D / 32; ++ch) {
-                    uint32_t v[32];
-                    tmem_ld32_wait(lane_base + col + ch * 32, v);
-                    if (kvrow < p.N) {
-                        uint4* d4 = reinterpret_cast<uint4*>(out + ch * 32);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            d4[e] = make_uint4(
-                                pack_bf16(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
-                                pack_bf16(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
-                                pack_bf16(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
-                                pack_bf16(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
-                    }
+                    for (int e = 0; e < 4; ++e)
+                        d4[e] = make_uint4(
+                            pack_bf16(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
+                            pack_bf16(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
+                            pack_bf16(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
+                            pack_bf16(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
                 }
             }
         }

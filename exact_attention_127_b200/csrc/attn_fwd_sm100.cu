@@ -1070,12 +1070,13 @@ int std_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
 
 #include "attn_bwd.cuh"
 
-/* Backward pass, host side.  Workspace: dQ accumulator (fp32 [BH, N, d]),
- * D and LSE*log2(e) (fp32 [BH, Np] each), 256-byte aligned pieces. */
+/* Backward pass, host side.  Workspace: the tiled dQ accumulator (fp32,
+ * BH * Np * d values), D and LSE*log2(e) (fp32 [BH, Np] each), 256-byte
+ * aligned pieces. */
 size_t bwd_ws_bytes(int64_t BH, int64_t N, int64_t d) {
     const int64_t Np = (N + BLOCK_M - 1) / BLOCK_M * BLOCK_M;
     auto a256 = [](size_t x) { return (x + 255u) & ~static_cast<size_t>(255u); };
-    return a256(static_cast<size_t>(BH) * N * d * 4) + 2 * a256(static_cast<size_t>(BH) * Np * 4);
+    return a256(static_cast<size_t>(BH) * Np * d * 4) + 2 * a256(static_cast<size_t>(BH) * Np * 4);
 }
 
 template <int D, bool CAUSAL>
@@ -1089,13 +1090,14 @@ int bwd_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
         return ATTN_ERR_LAUNCH;
     }
     const int64_t prows = static_cast<int64_t>(prm.BH) * prm.Np;
+    if (cudaMemsetAsync(prm.dq_acc, 0, static_cast<size_t>(prows) * D * 4, stream) != cudaSuccess)
+        return ATTN_ERR_CUDA;
     bwd_pre_kernel<D><<<static_cast<unsigned>((prows + 7) / 8), 256, 0, stream>>>(
-        o, dout, lse, const_cast<float*>(prm.Dp), const_cast<float*>(prm.lse2), prm.dq_acc, prm.N,
-        prm.Np, prm.BH);
+        o, dout, lse, const_cast<float*>(prm.Dp), const_cast<float*>(prm.lse2), prm.N, prm.Np,
+        prm.BH);
     kern<<<dim3(prm.nblk, prm.BH), BWD_THREADS, SMEM, stream>>>(mq, mk, mv, mdo, prm);
-    const int64_t n = static_cast<int64_t>(prm.BH) * prm.N * D;
-    bwd_post_kernel<<<static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 148 * 16)), 256, 0,
-                      stream>>>(prm.dq_acc, prm.dq, n);
+    bwd_post_kernel<D><<<static_cast<unsigned>(prm.BH * prm.nblk), BLOCK_M, 0, stream>>>(
+        prm.dq_acc, prm.dq, prm.N, prm.nblk);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
     return ATTN_OK;
 }
@@ -1135,7 +1137,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     prm.dk = static_cast<__nv_bfloat16*>(dk);
     prm.dv = static_cast<__nv_bfloat16*>(dv);
     prm.dq_acc = reinterpret_cast<float*>(ws);
-    prm.Dp = reinterpret_cast<float*>(ws + a256(static_cast<size_t>(BH) * N * d * 4));
+    prm.Dp = reinterpret_cast<float*>(ws + a256(static_cast<size_t>(BH) * Np * d * 4));
     prm.lse2 = prm.Dp + (a256(static_cast<size_t>(BH) * Np * 4) / 4);
     prm.N = static_cast<int>(N);
     prm.Np = static_cast<int>(Np);

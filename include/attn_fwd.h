@@ -103,8 +103,8 @@ int attn_device_status(void* stream, int reset);
 
 /*
  * attn_bwd_workspace_bytes -- device workspace attn_bwd needs: an fp32 dQ
- * accumulator [B, H, N, d] plus two fp32 [B, H, Np] vectors (Np = N rounded
- * up to 128), 256-byte aligned pieces.  0 for invalid or empty shapes.
+ * accumulator of B*H*Np*d values (Np = N rounded up to 128) plus two fp32
+ * [B, H, Np] vectors, 256-byte aligned pieces.  0 for invalid or empty shapes.
  */
 size_t attn_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
 
@@ -122,7 +122,7 @@ size_t attn_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
  *   workspace        : device, >= attn_bwd_workspace_bytes, 256-byte aligned,
  *                      caller-owned, contents ignored on entry; calls that
  *                      overlap on the GPU must not share it.
- * Three kernels are enqueued on `stream`.  Same d, scale, alignment and error
+ * A memset and three kernels are enqueued on `stream`.  Same d, scale, alignment and error
  * conventions as attn_fwd; additionally B*H <= 65535.
  */
 int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,

@@ -83,8 +83,13 @@ def load_peaks():
 
 
 def source_digest() -> str:
+    """sha256 of the forward pass's source: the part of the file before the
+    standard path and the backward pass are included (device helpers, the
+    kernel, its host-side launch and fwd_impl)."""
     with open(SRC, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()
+        text = f.read()
+    cut = text.find(b'#include "attn_standard.cuh"')
+    return hashlib.sha256(text[:cut] if cut >= 0 else text).hexdigest()
 
 
 def load_traffic(workload: str):

@@ -972,6 +972,55 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
     return ATTN_OK;
 }
 
+/* The forward call behind attn_fwd and the timeout test hook. */
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+             int64_t H, int64_t N, int64_t d, int causal, float scale, void* stream,
+             uint64_t wait_limit_ns, int withhold_kv) {
+    bool empty = false;
+    int st = validate_shape(B, H, N, d, scale, &empty);
+    if (st != ATTN_OK || empty) return st;
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
+    const void* ptrs[5] = {q, k, v, o, lse};
+    for (const void* ptr : ptrs)
+        if (reinterpret_cast<uintptr_t>(ptr) & 15u) return ATTN_ERR_ALIGN;
+    const size_t tbytes = static_cast<size_t>(B * H * N * d) * 2;
+    const size_t lbytes = static_cast<size_t>(B * H * N) * 4;
+    if (ranges_overlap(o, tbytes, q, tbytes) || ranges_overlap(o, tbytes, k, tbytes) ||
+        ranges_overlap(o, tbytes, v, tbytes) || ranges_overlap(lse, lbytes, q, tbytes) ||
+        ranges_overlap(lse, lbytes, k, tbytes) || ranges_overlap(lse, lbytes, v, tbytes) ||
+        ranges_overlap(lse, lbytes, o, tbytes))
+        return ATTN_ERR_OVERLAP;
+
+    int dev = 0;
+    DeviceInfo* di = nullptr;
+    if ((st = device_info(&dev, &di)) != ATTN_OK) return st;
+    EncodeTiledFn enc = nullptr;
+    if ((st = get_encode(&enc)) != ATTN_OK) return st;
+    const int64_t BH = B * H;
+    CUtensorMap mq, mk, mv;
+    if ((st = encode_map(enc, &mq, q, BH, N, d)) != ATTN_OK) return st;
+    if ((st = encode_map(enc, &mk, k, BH, N, d)) != ATTN_OK) return st;
+    if ((st = encode_map(enc, &mv, v, BH, N, d)) != ATTN_OK) return st;
+
+    FwdParams prm;
+    prm.o = static_cast<__nv_bfloat16*>(o);
+    prm.lse = lse;
+    prm.N = static_cast<int>(N);
+    prm.BH = static_cast<int>(BH);
+    prm.n_pairs = static_cast<int>((N + UNIT_ROWS - 1) / UNIT_ROWS);
+    prm.nkv = static_cast<int>((N + BLOCK_N - 1) / BLOCK_N);
+    prm.n_units = prm.BH * prm.n_pairs;
+    prm.scale_log2 = scale * LOG2E;
+    prm.wait_limit_ns = wait_limit_ns;
+    prm.withhold_kv = withhold_kv;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (d == 64)
+        return causal ? launch<64, true>(mq, mk, mv, prm, di, s) : launch<64, false>(mq, mk, mv, prm, di, s);
+    return causal ? launch<128, true>(mq, mk, mv, prm, di, s) : launch<128, false>(mq, mk, mv, prm, di, s);
+}
+
+/* Everything above is the forward pass; the standard path and the backward
+ * pass follow. */
 #include "attn_standard.cuh"
 
 /* The unfused three-kernel path (S and P through device memory), host side. */
@@ -1154,53 +1203,6 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
                       : bwd_launch<64, false>(mq, mk, mv, mdo, ob, db, lse, prm, s);
     return causal ? bwd_launch<128, true>(mq, mk, mv, mdo, ob, db, lse, prm, s)
                   : bwd_launch<128, false>(mq, mk, mv, mdo, ob, db, lse, prm, s);
-}
-
-/* The forward call behind attn_fwd and the timeout test hook. */
-int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
-             int64_t H, int64_t N, int64_t d, int causal, float scale, void* stream,
-             uint64_t wait_limit_ns, int withhold_kv) {
-    bool empty = false;
-    int st = validate_shape(B, H, N, d, scale, &empty);
-    if (st != ATTN_OK || empty) return st;
-    if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
-    const void* ptrs[5] = {q, k, v, o, lse};
-    for (const void* ptr : ptrs)
-        if (reinterpret_cast<uintptr_t>(ptr) & 15u) return ATTN_ERR_ALIGN;
-    const size_t tbytes = static_cast<size_t>(B * H * N * d) * 2;
-    const size_t lbytes = static_cast<size_t>(B * H * N) * 4;
-    if (ranges_overlap(o, tbytes, q, tbytes) || ranges_overlap(o, tbytes, k, tbytes) ||
-        ranges_overlap(o, tbytes, v, tbytes) || ranges_overlap(lse, lbytes, q, tbytes) ||
-        ranges_overlap(lse, lbytes, k, tbytes) || ranges_overlap(lse, lbytes, v, tbytes) ||
-        ranges_overlap(lse, lbytes, o, tbytes))
-        return ATTN_ERR_OVERLAP;
-
-    int dev = 0;
-    DeviceInfo* di = nullptr;
-    if ((st = device_info(&dev, &di)) != ATTN_OK) return st;
-    EncodeTiledFn enc = nullptr;
-    if ((st = get_encode(&enc)) != ATTN_OK) return st;
-    const int64_t BH = B * H;
-    CUtensorMap mq, mk, mv;
-    if ((st = encode_map(enc, &mq, q, BH, N, d)) != ATTN_OK) return st;
-    if ((st = encode_map(enc, &mk, k, BH, N, d)) != ATTN_OK) return st;
-    if ((st = encode_map(enc, &mv, v, BH, N, d)) != ATTN_OK) return st;
-
-    FwdParams prm;
-    prm.o = static_cast<__nv_bfloat16*>(o);
-    prm.lse = lse;
-    prm.N = static_cast<int>(N);
-    prm.BH = static_cast<int>(BH);
-    prm.n_pairs = static_cast<int>((N + UNIT_ROWS - 1) / UNIT_ROWS);
-    prm.nkv = static_cast<int>((N + BLOCK_N - 1) / BLOCK_N);
-    prm.n_units = prm.BH * prm.n_pairs;
-    prm.scale_log2 = scale * LOG2E;
-    prm.wait_limit_ns = wait_limit_ns;
-    prm.withhold_kv = withhold_kv;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (d == 64)
-        return causal ? launch<64, true>(mq, mk, mv, prm, di, s) : launch<64, false>(mq, mk, mv, prm, di, s);
-    return causal ? launch<128, true>(mq, mk, mv, prm, di, s) : launch<128, false>(mq, mk, mv, prm, di, s);
 }
 
 }  // namespace

@@ -8,12 +8,12 @@ log-sum-exp, for bf16 [B, H, N, d] CUDA tensors with d in {64, 128};
 attn_decode does the same for one new query row per head against N cached
 keys (split-K/V).
 """
-from ._lib import (AttnError, attn_bwd, attn_decode, attn_fwd, attn_fwd_host, attn_standard,
-                   bwd_workspace_bytes, decode_workspace_bytes, device_status, header_functions,
-                   host_workspace_bytes, load_library, standard_workspace_bytes, status_str,
-                   version)
+from ._lib import (AttnError, attn_bwd, attn_decode, attn_fwd, attn_fwd_fp8, attn_fwd_host,
+                   attn_standard, bwd_workspace_bytes, decode_workspace_bytes, device_status,
+                   fp8_workspace_bytes, header_functions, host_workspace_bytes, load_library,
+                   standard_workspace_bytes, status_str, version)
 
-__all__ = ["AttnError", "attn_bwd", "attn_decode", "attn_fwd", "attn_fwd_host", "attn_standard",
-           "bwd_workspace_bytes",
+__all__ = ["AttnError", "attn_bwd", "attn_decode", "attn_fwd", "attn_fwd_fp8", "attn_fwd_host",
+           "attn_standard", "bwd_workspace_bytes", "fp8_workspace_bytes",
            "decode_workspace_bytes", "device_status", "header_functions", "host_workspace_bytes",
            "load_library", "standard_workspace_bytes", "status_str", "version"]

@@ -62,6 +62,12 @@ def load_library():
     lib.attn_standard.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, c_int, ctypes.c_float,
                                   vp, ctypes.c_size_t, vp]
     lib.attn_standard.restype = c_int
+    lib.attn_fwd_fp8_workspace_bytes.argtypes = [i64, i64, i64, i64]
+    lib.attn_fwd_fp8_workspace_bytes.restype = ctypes.c_size_t
+    f32 = ctypes.c_float
+    lib.attn_fwd_fp8.argtypes = [vp, vp, vp, f32, f32, f32, vp, vp, i64, i64, i64, i64, c_int, f32,
+                                 vp, ctypes.c_size_t, vp]
+    lib.attn_fwd_fp8.restype = c_int
     lib.attn_decode_workspace_bytes.argtypes = [i64, i64, i64, i64]
     lib.attn_decode_workspace_bytes.restype = ctypes.c_size_t
     lib.attn_decode.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, ctypes.c_float, vp,
@@ -255,6 +261,48 @@ def attn_standard(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: boo
                                workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_standard")
+    return out, lse
+
+
+def fp8_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(load_library().attn_fwd_fp8_workspace_bytes(B, H, N, d))
+
+
+def attn_fwd_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_descale: float = 1.0,
+                 k_descale: float = 1.0, v_descale: float = 1.0, causal: bool = False,
+                 scale: float | None = None, out: torch.Tensor | None = None,
+                 lse: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                 stream=None):
+    """The forward pass on e4m3 inputs (torch.float8_e4m3fn [B, H, N, 128] CUDA
+    tensors): the scores use q8*q_descale and k8*k_descale, the values
+    v8*v_descale.  O (bf16) and LSE (fp32) as attn_fwd."""
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+        if t.dtype != torch.float8_e4m3fn:
+            raise ValueError(f"{name} must be float8_e4m3fn, got {t.dtype}")
+        if t.dim() != 4 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"{name} must be a contiguous CUDA [B, H, N, d] tensor")
+    if not (q8.shape == k8.shape == v8.shape) or not (q8.device == k8.device == v8.device):
+        raise ValueError("q8, k8, v8 must share one shape and device")
+    B, H, N, d = q8.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    if workspace is None:
+        workspace = torch.empty(max(fp8_workspace_bytes(B, H, N, d), 1), dtype=torch.uint8,
+                                device=q8.device)
+    lib = load_library()
+    with torch.cuda.device(q8.device):
+        rc = lib.attn_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), float(q_descale),
+                              float(k_descale), float(v_descale), out.data_ptr(), lse.data_ptr(),
+                              B, H, N, d, int(bool(causal)), float(scale), workspace.data_ptr(),
+                              workspace.numel(), _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_fp8")
     return out, lse
 
 

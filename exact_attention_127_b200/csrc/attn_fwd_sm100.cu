@@ -72,11 +72,13 @@ constexpr uint32_t WAIT_MAX_ITERS = 1u << 28;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float LOG2E = 1.4426950408889634f;
 
-template <int D>
+/* FP8: e4m3 Q, K, V (d = 128: one 128-byte swizzle atom per row), V read
+ * transposed (d rows, keys contiguous) so that every operand is K-major. */
+template <int D, bool FP8 = false>
 struct Cfg {
-    static constexpr int TILE_BYTES = BLOCK_M * D * 2;   // 128 rows x D bf16
-    static constexpr int CHUNKS = D / CHUNK_ELEMS;       // swizzle atoms along d
-    static constexpr int NSTAGE = (D == 128) ? 2 : 4;    // ring stages, each K_j then V_j
+    static constexpr int TILE_BYTES = BLOCK_M * D * (FP8 ? 1 : 2);   // 128 rows x D elements
+    static constexpr int CHUNKS = FP8 ? 1 : D / CHUNK_ELEMS;          // swizzle atoms along d
+    static constexpr int NSTAGE = (FP8 || D == 64) ? 4 : 2;  // ring stages, each K_j then V_j
     static constexpr int Q_OFF = 0;
     static constexpr int RING_OFF = 2 * TILE_BYTES;
     static constexpr int BAR_OFF = RING_OFF + 2 * NSTAGE * TILE_BYTES;
@@ -87,6 +89,7 @@ struct Cfg {
     static constexpr uint32_t S_COL0 = 0, S_COL1 = 128;
     static constexpr uint32_t O_COL0 = 256, O_COL1 = 256 + D;
     static_assert(D == 64 || D == 128, "head dim");
+    static_assert(!FP8 || D == 128, "e4m3 inputs: d = 128 only");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
@@ -101,6 +104,7 @@ struct FwdParams {
     float scale_log2;  // scale * log2(e)
     uint64_t wait_limit_ns;  // bound on every mbarrier wait
     int withhold_kv;         // test hook: the producer never loads K/V, so waits run out
+    float o_scale;           // e4m3 path: V's descale factor, applied to O at the end
 };
 
 __device__ int g_attn_status = 0;
@@ -271,6 +275,66 @@ __device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, 
     }
 }
 
+/* e4m3 x e4m3 -> fp32 (kind::f8f6f4), dense, both operands K-major.
+ * Bits: [4,6) D format (1 = f32), [7,10) / [10,13) A / B format (0 = E4M3),
+ * 15 / 16 majors (0 = K), [17,23) N >> 3, [24,29) M >> 4. */
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
+    return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+/* S = Q K^T with e4m3 Q and K, d = 128 (a row is one 128-byte swizzle atom):
+ * 4 MMAs with K = 32, each starting 32 bytes further. */
+__device__ __forceinline__ void issue_qk_f8(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc) {
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t off = static_cast<uint64_t>((kk * 32) >> 4);
+        mma_ss_f8(d_tmem, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
+    }
+}
+
+/* O += P V for keys [64*half, 64*half + 64) with e4m3 P and V: 2 MMAs with
+ * K = 32.  P is in TMEM (keys 4c .. 4c+3 in column c, key 4c in bits 0-7); b0
+ * describes V^T (d rows, keys contiguous: K-major), 32 keys = 32 bytes further
+ * per k-step. */
+__device__ __forceinline__ void issue_pv_half_f8(uint32_t d_tmem, uint32_t p_tmem, uint64_t b0,
+                                                 uint32_t idesc, uint32_t acc_first, int half) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int kk = half * 2 + i;
+        mma_ts_f8(d_tmem, p_tmem + kk * 8, b0 + static_cast<uint64_t>((kk * 32) >> 4), idesc,
+                  (i > 0) ? 1u : acc_first);
+    }
+}
+
+template <int D, bool FP8>
+__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc) {
+    if constexpr (FP8) issue_qk_f8(d_tmem, a0, b0, idesc);
+    else issue_qk<D>(d_tmem, a0, b0, idesc);
+}
+
+template <bool FP8>
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t b0,
+                                         uint32_t idesc, uint32_t acc_first, int half) {
+    if constexpr (FP8) issue_pv_half_f8(d_tmem, p_tmem, b0, idesc, acc_first, half);
+    else issue_pv_half(d_tmem, p_tmem, b0, idesc, acc_first, half);
+}
+
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -355,6 +419,18 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return r;
 }
 
+/* Four fp32 -> four e4m3 in one word, round to nearest even, saturating at
+ * +-448; `a` in bits 0-7.  (cvt ... e4m3x2 d, x, y puts x in the upper byte.) */
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(r) : "f"(a), "f"(b), "f"(c), "f"(d));
+    return r;
+}
+
 /* tcgen05.ld of 128 consecutive 32-bit columns of this thread's TMEM lane, with
  * the wait in the same asm statement so no use of v[] can be scheduled early. */
 __device__ __forceinline__ void tmem_ld128_wait(uint32_t taddr, uint32_t* v) {
@@ -435,6 +511,16 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
         : "memory");
 }
 
+/* tcgen05.st of 8 consecutive 32-bit columns into this thread's TMEM lane. */
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+        :
+        : "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]),
+          "r"(v[6]), "r"(v[7])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -485,12 +571,12 @@ __device__ __forceinline__ int unit_index(int round) {
 /* ------------------------------------------------------------------------ */
 /* The kernel                                                                */
 /* ------------------------------------------------------------------------ */
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool FP8 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-    using C = Cfg<D>;
+    using C = Cfg<D, FP8>;
     constexpr int NSTAGE = C::NSTAGE;
     constexpr uint32_t TILE = C::TILE_BYTES;
 
@@ -582,10 +668,15 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     }
                     mbar_arrive_expect_tx(bar_kv_full(s), 2 * TILE);
                     for (int kv = 0; kv < 2; ++kv)
-                        for (int c = 0; c < C::CHUNKS; ++c)
-                            tma_load_3d(kv ? &tm_v : &tm_k,
-                                        sRing + (2 * s + kv) * TILE + c * CHUNK_BYTES,
-                                        bar_kv_full(s), c * CHUNK_ELEMS, j * BLOCK_N, u.bh);
+                        for (int c = 0; c < C::CHUNKS; ++c) {
+                            if (FP8 && kv)   // V^T: rows are d, keys run along x
+                                tma_load_3d(&tm_v, sRing + (2 * s + 1) * TILE, bar_kv_full(s),
+                                            j * BLOCK_N, 0, u.bh);
+                            else
+                                tma_load_3d(kv ? &tm_v : &tm_k,
+                                            sRing + (2 * s + kv) * TILE + c * CHUNK_BYTES,
+                                            bar_kv_full(s), c * CHUNK_ELEMS, j * BLOCK_N, u.bh);
+                        }
                     ++it;
                 }
                 ++local;
@@ -612,15 +703,17 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
          * Waits on TMA barriers need no tcgen05 fence (no tcgen05 op precedes
          * their arrival); waits on softmax barriers do. */
         if (lane == 0) {
-            constexpr uint32_t IDESC_S = idesc_bf16(BLOCK_M, BLOCK_N, false);
-            constexpr uint32_t IDESC_PV = idesc_bf16(BLOCK_M, D, true);
+            constexpr uint32_t IDESC_S = FP8 ? idesc_e4m3(BLOCK_M, BLOCK_N)
+                                             : idesc_bf16(BLOCK_M, BLOCK_N, false);
+            constexpr uint32_t IDESC_PV = FP8 ? idesc_e4m3(BLOCK_M, D) : idesc_bf16(BLOCK_M, D, true);
             constexpr uint64_t SLOT_STEP = TILE >> 4;       // descriptor units per ring slot
             const uint32_t ts0 = tmem + C::S_COL0, ts1 = tmem + C::S_COL1;
             const uint32_t to0 = tmem + C::O_COL0, to1 = tmem + C::O_COL1;
             const uint64_t qd0 = sdesc_sw128(sQ[0], 16, 1024);
             const uint64_t qd1 = sdesc_sw128(sQ[1], 16, 1024);
             const uint64_t kd_base = sdesc_sw128(sRing, 16, 1024);                    // K-major
-            const uint64_t vd_base = sdesc_sw128(sRing + TILE, CHUNK_BYTES, 1024);    // MN-major
+            const uint64_t vd_base = FP8 ? sdesc_sw128(sRing + TILE, 16, 1024)        // V^T, K-major
+                                         : sdesc_sw128(sRing + TILE, CHUNK_BYTES, 1024);  // MN-major
             const uint32_t bs0 = bar_s_full0, bs1 = bar_s_full0 + 8;
             const uint32_t bh0 = bar_p_half0, bh1 = bar_p_half0 + 8;
             const uint32_t bp0 = bar_p_ready0, bp1 = bar_p_ready0 + 8;
@@ -641,8 +734,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const uint32_t st = it % NSTAGE;
                     if (!mbar_wait(bar_kv_full(st), (it / NSTAGE) & 1u, abort_flag, wlim)) { aborted = true; break; }
                     const uint64_t kd = kd_base + 2 * st * SLOT_STEP;
-                    if (n0 > 0) { issue_qk<D>(ts0, qd0, kd, IDESC_S); mma_commit(bs0); }
-                    if (n1 > 0) { issue_qk<D>(ts1, qd1, kd, IDESC_S); mma_commit(bs1); }
+                    if (n0 > 0) { issue_s<D, FP8>(ts0, qd0, kd, IDESC_S); mma_commit(bs0); }
+                    if (n1 > 0) { issue_s<D, FP8>(ts1, qd1, kd, IDESC_S); mma_commit(bs1); }
                     if (nmax == 1) mma_commit(bar_q_empty);
                 }
                 for (int j = 0; j < nmax; ++j) {
@@ -655,11 +748,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     if (j < n0) {
                         if (!mbar_wait(bh0, pr0 & 1u, abort_flag, wlim)) { aborted = true; break; }
                         tc_fence_after();
-                        issue_pv_half(to0, ts0, vd, IDESC_PV, acc, 0);
+                        issue_pv<FP8>(to0, ts0, vd, IDESC_PV, acc, 0);
                         if (!mbar_wait(bp0, pr0 & 1u, abort_flag, wlim)) { aborted = true; break; }
                         ++pr0;
                         tc_fence_after();
-                        issue_pv_half(to0, ts0, vd, IDESC_PV, 1u, 1);
+                        issue_pv<FP8>(to0, ts0, vd, IDESC_PV, 1u, 1);
                         if (j == n0 - 1) mma_commit(bo0);
                     }
                     if (has_next &&
@@ -667,20 +760,20 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                         aborted = true;
                         break;
                     }
-                    if (j + 1 < n0) { issue_qk<D>(ts0, qd0, kd, IDESC_S); mma_commit(bs0); }
+                    if (j + 1 < n0) { issue_s<D, FP8>(ts0, qd0, kd, IDESC_S); mma_commit(bs0); }
                     if (j < n1) {
                         if (!mbar_wait(bh1, pr1 & 1u, abort_flag, wlim)) { aborted = true; break; }
                         tc_fence_after();
-                        issue_pv_half(to1, ts1, vd, IDESC_PV, acc, 0);
+                        issue_pv<FP8>(to1, ts1, vd, IDESC_PV, acc, 0);
                         if (!mbar_wait(bp1, pr1 & 1u, abort_flag, wlim)) { aborted = true; break; }
                         ++pr1;
                         tc_fence_after();
-                        issue_pv_half(to1, ts1, vd, IDESC_PV, 1u, 1);
+                        issue_pv<FP8>(to1, ts1, vd, IDESC_PV, 1u, 1);
                         if (j == n1 - 1) mma_commit(bo1);
                     }
                     mma_commit(bar_kv_empty(st));                    // K_j and V_j read
                     ++it;
-                    if (j + 1 < n1) { issue_qk<D>(ts1, qd1, kd, IDESC_S); mma_commit(bs1); }
+                    if (j + 1 < n1) { issue_s<D, FP8>(ts1, qd1, kd, IDESC_S); mma_commit(bs1); }
                     if (j + 1 == nmax - 1) mma_commit(bar_q_empty);  // last S of the unit issued
                 }
                 ++local;
@@ -768,6 +861,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                 for (int qtr = 0; qtr < 4; ++qtr) {
                     const int half = qtr >> 1;
                     uint32_t pk[BLOCK_N / 8];
+                    float pq[FP8 ? BLOCK_N / 4 : 1];
 #pragma unroll
                     for (int k = 0; k < BLOCK_N / 8; ++k) {
                         const int cc = qtr * (BLOCK_N / 4) + 2 * k;
@@ -782,9 +876,22 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                         }
                         sum_a += p0;
                         sum_b += p1;
-                        pk[k] = pack_bf16(p0, p1);
+                        if constexpr (FP8) {
+                            pq[2 * k] = p0;
+                            pq[2 * k + 1] = p1;
+                        } else {
+                            pk[k] = pack_bf16(p0, p1);
+                        }
                     }
-                    tmem_st16(s_addr + qtr * (BLOCK_N / 8), pk);
+                    if constexpr (FP8) {
+                        uint32_t p8[BLOCK_N / 16];
+#pragma unroll
+                        for (int e = 0; e < BLOCK_N / 16; ++e)
+                            p8[e] = pack_e4m3x4(pq[4 * e], pq[4 * e + 1], pq[4 * e + 2], pq[4 * e + 3]);
+                        tmem_st8(s_addr + qtr * (BLOCK_N / 16), p8);
+                    } else {
+                        tmem_st16(s_addr + qtr * (BLOCK_N / 8), pk);
+                    }
                     if (!warp_rescale && (qtr & 1)) {
                         tmem_wait_st();
                         tc_fence_before();
@@ -816,7 +923,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
+            float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
+            if constexpr (FP8) inv_l *= p.o_scale;
             const bool live = row < p.N;
             __nv_bfloat16* orow = p.o + (static_cast<size_t>(u.bh) * p.N + (live ? row : 0)) * D;
 #pragma unroll
@@ -867,7 +975,7 @@ struct DeviceInfo {
     bool ready = false;
     int status = ATTN_OK;   // ATTN_ERR_DEVICE when the device is not CC 10.0
     int num_sms = 0;
-    bool smem_set[4] = {false, false, false, false};
+    bool smem_set[8] = {false, false, false, false, false, false, false, false};
 };
 
 std::mutex g_mutex;
@@ -949,12 +1057,12 @@ int validate_shape(int64_t B, int64_t H, int64_t N, int64_t d, float scale, bool
     return ATTN_OK;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool FP8 = false>
 int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
            const FwdParams& prm, DeviceInfo* di, cudaStream_t stream) {
-    auto kern = attn_fwd_sm100_kernel<D, CAUSAL>;
-    constexpr int SMEM = Cfg<D>::SMEM_BYTES;
-    const int key = (D == 128 ? 2 : 0) + (CAUSAL ? 1 : 0);
+    auto kern = attn_fwd_sm100_kernel<D, CAUSAL, FP8>;
+    constexpr int SMEM = Cfg<D, FP8>::SMEM_BYTES;
+    const int key = (FP8 ? 4 : 0) + (D == 128 ? 2 : 0) + (CAUSAL ? 1 : 0);
     {
         std::lock_guard<std::mutex> lock(g_mutex);
         if (!di->smem_set[key]) {
@@ -1013,10 +1121,129 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     prm.scale_log2 = scale * LOG2E;
     prm.wait_limit_ns = wait_limit_ns;
     prm.withhold_kv = withhold_kv;
+    prm.o_scale = 1.0f;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (d == 64)
         return causal ? launch<64, true>(mq, mk, mv, prm, di, s) : launch<64, false>(mq, mk, mv, prm, di, s);
     return causal ? launch<128, true>(mq, mk, mv, prm, di, s) : launch<128, false>(mq, mk, mv, prm, di, s);
+}
+
+/* ------------------------------------------------------------------------ */
+/* e4m3 inputs: V transposed into the workspace, then the same kernel        */
+/* ------------------------------------------------------------------------ */
+/* V [BH, N, 128] e4m3 -> V^T [BH, 128, Np] (Np = N rounded up to 128; keys
+ * past N are zero, so masked keys multiply zeros).  One CTA per (head, block
+ * of 128 keys), through a shared-memory tile; 16-byte loads and stores. */
+__global__ void __launch_bounds__(256)
+fp8_transpose_v_kernel(const uint8_t* __restrict__ v, uint8_t* __restrict__ vt, int N, int Np) {
+    __shared__ uint8_t tile[128][128 + 4];
+    const int kb = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
+    const uint8_t* src = v + (static_cast<int64_t>(bh) * N + static_cast<int64_t>(kb) * 128) * 128;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int unit = t + 256 * i;              // 128 keys x 8 units of 16 bytes
+        const int key = unit >> 3, c = unit & 7;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (kb * 128 + key < N) val = *reinterpret_cast<const uint4*>(src + key * 128 + c * 16);
+        const uint32_t w[4] = {val.x, val.y, val.z, val.w};
+#pragma unroll
+        for (int b = 0; b < 16; ++b) tile[key][c * 16 + b] = static_cast<uint8_t>(w[b >> 2] >> (8 * (b & 3)));
+    }
+    __syncthreads();
+    uint8_t* dst = vt + static_cast<int64_t>(bh) * 128 * Np + static_cast<int64_t>(kb) * 128;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int unit = t + 256 * i;              // 128 d rows x 8 units of 16 keys
+        const int row = unit >> 3, c = unit & 7;
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int b = 0; b < 16; ++b) w[b >> 2] |= static_cast<uint32_t>(tile[c * 16 + b][row]) << (8 * (b & 3));
+        *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(row) * Np + c * 16) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+/* 3-D map over 8-bit data [BH][rows][inner], box 128 x 128 bytes, 128B swizzle. */
+int encode_map_u8(EncodeTiledFn fn, CUtensorMap* map, const void* ptr, int64_t BH, int64_t rows,
+                  int64_t inner) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
+                          static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows * inner)};
+    cuuint32_t box[3] = {128, BLOCK_M, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+size_t fp8_ws_bytes(int64_t BH, int64_t N) {
+    const int64_t Np = (N + BLOCK_N - 1) / BLOCK_N * BLOCK_N;
+    return static_cast<size_t>(BH) * 128 * Np;
+}
+
+int fp8_impl(const void* q, const void* k, const void* v, float q_descale, float k_descale,
+             float v_descale, void* o, float* lse, int64_t B, int64_t H, int64_t N, int64_t d,
+             int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+    bool empty = false;
+    int st = validate_shape(B, H, N, d, scale, &empty);
+    if (st != ATTN_OK) return st;
+    if (d != 128) return ATTN_ERR_HEADDIM;
+    if (empty) return ATTN_OK;
+    if (B * H > 65535) return ATTN_ERR_SHAPE;
+    const float ds[3] = {q_descale, k_descale, v_descale};
+    for (float x : ds)
+        if (!(x > 0.0f) || !isfinite(x)) return ATTN_ERR_SCALE;
+    if (!isfinite(scale * q_descale * k_descale * LOG2E)) return ATTN_ERR_SCALE;
+    const void* ptrs[5] = {q, k, v, o, lse};
+    for (const void* ptr : ptrs) {
+        if (!ptr) return ATTN_ERR_NULL;
+        if (reinterpret_cast<uintptr_t>(ptr) & 15u) return ATTN_ERR_ALIGN;
+    }
+    const int64_t BH = B * H;
+    const size_t ws_need = fp8_ws_bytes(BH, N);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < ws_need)
+        return ATTN_ERR_WORKSPACE;
+    const size_t in_bytes = static_cast<size_t>(BH * N * d);
+    const size_t obytes = in_bytes * 2, lbytes = static_cast<size_t>(BH * N) * 4;
+    const void* ins[3] = {q, k, v};
+    for (const void* in : ins)
+        if (ranges_overlap(o, obytes, in, in_bytes) || ranges_overlap(lse, lbytes, in, in_bytes) ||
+            ranges_overlap(workspace, ws_need, in, in_bytes))
+            return ATTN_ERR_OVERLAP;
+    if (ranges_overlap(o, obytes, lse, lbytes) || ranges_overlap(workspace, ws_need, o, obytes) ||
+        ranges_overlap(workspace, ws_need, lse, lbytes))
+        return ATTN_ERR_OVERLAP;
+    int dev = 0;
+    DeviceInfo* di = nullptr;
+    if ((st = device_info(&dev, &di)) != ATTN_OK) return st;
+    EncodeTiledFn enc = nullptr;
+    if ((st = get_encode(&enc)) != ATTN_OK) return st;
+    const int64_t Np = (N + BLOCK_N - 1) / BLOCK_N * BLOCK_N;
+    CUtensorMap mq, mk, mvt;
+    if ((st = encode_map_u8(enc, &mq, q, BH, N, d)) != ATTN_OK) return st;
+    if ((st = encode_map_u8(enc, &mk, k, BH, N, d)) != ATTN_OK) return st;
+    if ((st = encode_map_u8(enc, &mvt, workspace, BH, d, Np)) != ATTN_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    fp8_transpose_v_kernel<<<dim3(static_cast<unsigned>(Np / BLOCK_N), static_cast<unsigned>(BH)),
+                             256, 0, s>>>(static_cast<const uint8_t*>(v),
+                                          static_cast<uint8_t*>(workspace), static_cast<int>(N),
+                                          static_cast<int>(Np));
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+    FwdParams prm;
+    prm.o = static_cast<__nv_bfloat16*>(o);
+    prm.lse = lse;
+    prm.N = static_cast<int>(N);
+    prm.BH = static_cast<int>(BH);
+    prm.n_pairs = static_cast<int>((N + UNIT_ROWS - 1) / UNIT_ROWS);
+    prm.nkv = static_cast<int>(Np / BLOCK_N);
+    prm.n_units = prm.BH * prm.n_pairs;
+    prm.scale_log2 = scale * q_descale * k_descale * LOG2E;
+    prm.wait_limit_ns = WAIT_LIMIT_NS;
+    prm.withhold_kv = 0;
+    prm.o_scale = v_descale;
+    return causal ? launch<128, true, true>(mq, mk, mvt, prm, di, s)
+                  : launch<128, false, true>(mq, mk, mvt, prm, di, s);
 }
 
 /* Everything above is the forward pass; the standard path and the backward
@@ -1217,6 +1444,20 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
 int attn_fwd_test_wait_timeout(const void* q, const void* k, const void* v, void* o, float* lse,
                                int64_t B, int64_t H, int64_t N, int64_t d, void* stream) {
     return fwd_impl(q, k, v, o, lse, B, H, N, d, 0, 0.125f, stream, TEST_WAIT_LIMIT_NS, 1);
+}
+
+size_t attn_fwd_fp8_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {
+    bool empty = false;
+    if (validate_shape(B, H, N, d, 1.0f, &empty) != ATTN_OK || empty || d != 128 || B * H > 65535)
+        return 0;
+    return fp8_ws_bytes(B * H, N);
+}
+
+int attn_fwd_fp8(const void* q, const void* k, const void* v, float q_descale, float k_descale,
+                 float v_descale, void* o, float* lse, int64_t B, int64_t H, int64_t N, int64_t d,
+                 int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+    return fp8_impl(q, k, v, q_descale, k_descale, v_descale, o, lse, B, H, N, d, causal, scale,
+                    workspace, workspace_bytes, stream);
 }
 
 size_t attn_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {

@@ -89,6 +89,19 @@ def make_qkv(B: int, H: int, N: int, d: int, seed: int, qk_std: float = 1.0,
     return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
 
 
+def make_qkv_e4m3(B: int, H: int, N: int, d: int, seed: int, amplitude: float = 1.0,
+                  descale: float = 1.0):
+    """Seeded e4m3 (torch.float8_e4m3fn) CPU tensors for the 8-bit forward:
+    make_qkv's bf16 draws times `amplitude`, divided by `descale` and rounded
+    to e4m3 (nearest even).  The attention they stand for is that of
+    x8 * descale, which is exact in fp64."""
+    out = []
+    for t in make_qkv(B, H, N, d, seed):
+        x = t.float() * float(amplitude) / float(descale)
+        out.append(x.to(torch.float8_e4m3fn))
+    return tuple(out)
+
+
 @dataclass(frozen=True)
 class DecodeWorkload:
     """One new query row per head against N cached keys (decode)."""

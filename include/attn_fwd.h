@@ -152,6 +152,36 @@ int attn_standard(const void* q, const void* k, const void* v, void* o, float* l
                   void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * attn_fwd_fp8_workspace_bytes -- device workspace attn_fwd_fp8 needs: V
+ * transposed, B*H*128*Np bytes (Np = N rounded up to 128).  0 for invalid or
+ * empty shapes and for d != 128.
+ */
+size_t attn_fwd_fp8_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
+
+/*
+ * attn_fwd_fp8 -- the fused forward pass on 8-bit inputs, the FP8 line of the
+ * Hopper-era design ("GPU 学习日报 Day 21", section 6): both GEMMs run on the
+ * tensor cores with e4m3 operands (tcgen05 kind::f8f6f4) and fp32 accumulators;
+ * the softmax and its statistics stay fp32, and P is rounded to e4m3 for P V.
+ *   q, k, v : device, e4m3 (OCP FP8 E4M3, 1 byte) [B, H, N, d], read only.  The
+ *             attention is that of q*q_descale, k*k_descale, v*v_descale.
+ *   q_descale, k_descale, v_descale : finite, > 0 (else ATTN_ERR_SCALE).
+ *   o       : device, bf16 [B, H, N, d], written.
+ *   lse     : device, fp32 [B, H, N], written (natural log, as attn_fwd).
+ *   workspace : device, >= attn_fwd_fp8_workspace_bytes, 256-byte aligned,
+ *             caller-owned, contents ignored on entry; it must not overlap the
+ *             inputs or outputs (ATTN_ERR_OVERLAP), and calls that overlap on
+ *             the GPU must not share it.
+ * d must be 128 (ATTN_ERR_HEADDIM otherwise); B*H <= 65535.  Two kernels are
+ * enqueued on `stream` (V transposed into the workspace, then the forward
+ * kernel).  Otherwise the conventions of attn_fwd.  Rounding P to e4m3 (3
+ * mantissa bits) makes |dO| up to 2^-4 * max_j |v_j| per element of O.
+ */
+int attn_fwd_fp8(const void* q, const void* k, const void* v, float q_descale, float k_descale,
+                 float v_descale, void* o, float* lse, int64_t B, int64_t H, int64_t N, int64_t d,
+                 int causal, float scale, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * attn_decode_workspace_bytes -- device workspace attn_decode needs for a shape
  * (the per-split partial results).  Returns 0 for invalid or empty shapes.
  */

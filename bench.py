@@ -464,6 +464,76 @@ def run_backward(args, w):
     return 0
 
 
+FP8_METRIC = "attention fwd TFLOP/s, e4m3 inputs (fp32 accumulate, e4m3 P)"
+FP8_OVER_BF16 = 2.0   # nominal dense e4m3 : bf16 tensor rate (4.5 : 2.25 PFLOP/s)
+
+
+def run_fp8(args, w):
+    """One step = one attn_fwd_fp8 call (V transposed into the workspace, then
+    the fused kernel on e4m3 operands) on a d = 128 forward workload."""
+    import torch
+
+    import exact_attention_127_b200 as attn
+
+    rank, local, world = dist_env()
+    if world > 1:
+        raise SystemExit("--dtype e4m3 runs on one GPU")
+    if w.d != 128:
+        raise SystemExit("--dtype e4m3 needs a d = 128 workload")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    attn.load_library()
+    q8, k8, v8 = (t.to(dev) for t in _inputs.make_qkv_e4m3(w.B, w.H, w.N, w.d, seed=w.seed))
+    o = torch.empty(q8.shape, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    ws = torch.empty(attn.fp8_workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.synchronize(dev)
+
+    def step():
+        attn.attn_fwd_fp8(q8, k8, v8, causal=w.causal, scale=w.scale, out=o, lse=lse,
+                          workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    sampler.start()
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            step()
+    e1.record(stream)
+    stream.synchronize()
+    sampler.stop()
+    if attn.device_status(reset=True, stream=stream) != 0:
+        raise RuntimeError("device-side error in the e4m3 forward")
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = w.flops()
+    peaks, peak_src = load_peaks()
+    peak = FP8_OVER_BF16 * peaks["bf16_tflops"]
+    tf = flops / (ms * 1e-3) / 1e12
+    cfg = config_of(w, 1)
+    cfg["inputs"] = "e4m3 (make_qkv's N(0,1) draws rounded to nearest), descales 1"
+    line = {
+        "metric": FP8_METRIC, "value": tf, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3", "data": "synthetic", "config": cfg,
+        "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tf / peak, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 dense matmul, burst (MEASURED_PEAKS.json), "
+                                    f"x {FP8_OVER_BF16:g} (nominal e4m3 : bf16 dense rate)",
+                     "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
+                     "kernel": "fp8_transpose_v_kernel + attn_fwd_sm100_kernel<128, causal, e4m3>",
+                     "algorithmic_flops_per_launch": flops},
+        "e2e": None, "gpu_launches": 2 * args.steps, "clocks": sampler.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_standard(args, w):
     """The unfused three-kernel path on a forward workload (context for the
     fused kernel): same metric (useful TFLOP/s); its roofline is HBM, since the
@@ -629,6 +699,8 @@ def main(argv=None):
     ap.add_argument("--ref-step-seconds", type=float, default=2.0)
     ap.add_argument("--ref-budget-seconds", type=float, default=150.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dtype", default="bf16", choices=["bf16", "e4m3"],
+                    help="forward operand type: bf16 (default) or e4m3 (attn_fwd_fp8, d = 128)")
     ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
                     help="forward (default) or the backward pass of the workload")
     ap.add_argument("--path", default="fused", choices=["fused", "standard"],
@@ -657,6 +729,8 @@ def main(argv=None):
         return run_reference(args, w)
     if args.pass_ == "bwd":
         return run_backward(args, w)
+    if args.dtype == "e4m3":
+        return run_fp8(args, w)
     if args.path == "standard":
         return run_standard(args, w)
     return run_cuda(args, w)

@@ -1133,33 +1133,55 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
 /* ------------------------------------------------------------------------ */
 /* V [BH, N, 128] e4m3 -> V^T [BH, 128, Np] (Np = N rounded up to 128; keys
  * past N are zero, so masked keys multiply zeros).  One CTA per (head, block
- * of 128 keys), through a shared-memory tile; 16-byte loads and stores. */
+ * of 128 keys).  A thread reads four keys x 16 bytes, transposes the 4 x 4
+ * byte blocks in registers and parks 32-bit words (4 keys of one column) in
+ * shared memory; the CTA then writes the block's 128 rows of V^T with
+ * 16-byte stores. */
+__device__ __forceinline__ void transpose4x4_bytes(const uint32_t w[4], uint32_t out[4]) {
+    // out[c] = byte c of w[0], w[1], w[2], w[3] (w[r] in byte r)
+    const uint32_t lo01 = __byte_perm(w[0], w[1], 0x5140), hi01 = __byte_perm(w[0], w[1], 0x7362);
+    const uint32_t lo23 = __byte_perm(w[2], w[3], 0x5140), hi23 = __byte_perm(w[2], w[3], 0x7362);
+    out[0] = __byte_perm(lo01, lo23, 0x5410);
+    out[1] = __byte_perm(lo01, lo23, 0x7632);
+    out[2] = __byte_perm(hi01, hi23, 0x5410);
+    out[3] = __byte_perm(hi01, hi23, 0x7632);
+}
+
 __global__ void __launch_bounds__(256)
 fp8_transpose_v_kernel(const uint8_t* __restrict__ v, uint8_t* __restrict__ vt, int N, int Np) {
-    __shared__ uint8_t tile[128][128 + 4];
+    __shared__ uint32_t tw[128][33];          // [column][group of 4 keys], padded row
     const int kb = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
     const uint8_t* src = v + (static_cast<int64_t>(bh) * N + static_cast<int64_t>(kb) * 128) * 128;
+    {
+        const int g = t >> 3, c16 = t & 7;    // keys 4g .. 4g+3, columns 16 c16 .. 16 c16 + 15
+        uint4 rows[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int unit = t + 256 * i;              // 128 keys x 8 units of 16 bytes
-        const int key = unit >> 3, c = unit & 7;
-        uint4 val = make_uint4(0u, 0u, 0u, 0u);
-        if (kb * 128 + key < N) val = *reinterpret_cast<const uint4*>(src + key * 128 + c * 16);
-        const uint32_t w[4] = {val.x, val.y, val.z, val.w};
+        for (int r = 0; r < 4; ++r) {
+            const int key = 4 * g + r;
+            rows[r] = make_uint4(0u, 0u, 0u, 0u);
+            if (kb * 128 + key < N)
+                rows[r] = *reinterpret_cast<const uint4*>(src + key * 128 + c16 * 16);
+        }
 #pragma unroll
-        for (int b = 0; b < 16; ++b) tile[key][c * 16 + b] = static_cast<uint8_t>(w[b >> 2] >> (8 * (b & 3)));
+        for (int wi = 0; wi < 4; ++wi) {
+            const uint32_t w[4] = {wi == 0 ? rows[0].x : wi == 1 ? rows[0].y : wi == 2 ? rows[0].z : rows[0].w,
+                                   wi == 0 ? rows[1].x : wi == 1 ? rows[1].y : wi == 2 ? rows[1].z : rows[1].w,
+                                   wi == 0 ? rows[2].x : wi == 1 ? rows[2].y : wi == 2 ? rows[2].z : rows[2].w,
+                                   wi == 0 ? rows[3].x : wi == 1 ? rows[3].y : wi == 2 ? rows[3].z : rows[3].w};
+            uint32_t out[4];
+            transpose4x4_bytes(w, out);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) tw[c16 * 16 + wi * 4 + cc][g] = out[cc];
+        }
     }
     __syncthreads();
     uint8_t* dst = vt + static_cast<int64_t>(bh) * 128 * Np + static_cast<int64_t>(kb) * 128;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int unit = t + 256 * i;              // 128 d rows x 8 units of 16 keys
-        const int row = unit >> 3, c = unit & 7;
-        uint32_t w[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-        for (int b = 0; b < 16; ++b) w[b >> 2] |= static_cast<uint32_t>(tile[c * 16 + b][row]) << (8 * (b & 3));
-        *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(row) * Np + c * 16) =
-            make_uint4(w[0], w[1], w[2], w[3]);
+        const int item = t + 256 * i;         // 128 columns x 8 runs of 16 keys
+        const int col = item >> 3, u = item & 7;
+        *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(col) * Np + u * 16) =
+            make_uint4(tw[col][4 * u], tw[col][4 * u + 1], tw[col][4 * u + 2], tw[col][4 * u + 3]);
     }
 }
 

@@ -44,12 +44,13 @@ def _grads(q, k, v, dout, causal, scale):
     return dq.cpu(), dk.cpu(), dv.cpu()
 
 
-def _check(q, k, v, dout, causal, scale, label):
+def _check(q, k, v, dout, causal, scale, label, heads=None):
     B, H, N, d = q.shape
+    heads = list(range(B * H)) if heads is None else list(heads)
     got = _grads(q, k, v, dout, causal, scale)
-    ref = oracle.attention_backward(q, k, v, dout, causal, scale)
+    ref = oracle.attention_backward(q, k, v, dout, causal, scale, heads=heads)
     for name, g, r in zip(("dq", "dk", "dv"), got, ref):
-        gf = g.reshape(B * H, N, d).double().numpy()
+        gf = g.reshape(B * H, N, d)[heads].double().numpy()
         err = np.abs(gf - r)
         rel = np.linalg.norm(gf - r) / max(np.linalg.norm(r), 1e-30)
         msg = f"{label} {name}: relL2={rel:.3e} max|err|={err.max():.3e} max|ref|={np.abs(r).max():.3e}"
@@ -79,6 +80,18 @@ def test_backward_larger_causal_two_heads():
     q, k, v = inputs.make_qkv(1, 2, 2048, 128, seed=41)
     dout = inputs.make_qkv(1, 2, 2048, 128, seed=42)[0]
     _check(q, k, v, dout, True, 1 / math.sqrt(128), "N=2048 d=128 causal")
+
+
+@pytest.mark.gpu
+def test_backward_headline_workload_two_heads():
+    """The configuration bench.py --pass bwd times (B=4, H=16, N=8192, d=128,
+    causal, the same dO), checked in full on the first and the last head."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    w = inputs.WORKLOADS[inputs.HEADLINE]
+    q, k, v = inputs.workload_inputs(w)
+    dout = inputs.make_qkv(w.B, w.H, w.N, w.d, w.seed + 100)[0]
+    _check(q, k, v, dout, w.causal, w.scale, w.name, heads=[0, w.B * w.H - 1])
 
 
 @pytest.mark.gpu

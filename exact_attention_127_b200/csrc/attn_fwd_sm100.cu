@@ -59,7 +59,14 @@ namespace {
 constexpr int BLOCK_M = 128;          // query rows per Q tile = TMEM lanes
 constexpr int BLOCK_N = 128;          // key/value rows per K/V block
 constexpr int UNIT_ROWS = 2 * BLOCK_M;  // a work unit = two Q tiles
-constexpr int NUM_THREADS = 320;
+constexpr int NUM_THREADS = 384;      // 3 warpgroups: softmax tile 0, softmax tile 1, TMA + MMA
+/* Register split (setmaxnreg): the kernel launches with 168 registers per
+ * thread (384 x 168 = 64512); the producer/MMA warpgroup gives back down to
+ * 88 so that the two softmax warpgroups can hold 208: 2*128*208 + 128*88 =
+ * 64512, exactly what the launch holds (a larger sum would wait forever). */
+constexpr int SOFTMAX_REGS = 208;
+constexpr int OTHER_REGS = 88;
+static_assert(2 * 128 * SOFTMAX_REGS + 128 * OTHER_REGS == NUM_THREADS * 168, "register split");
 constexpr int LOAD_WARP = 8;
 constexpr int MMA_WARP = 9;
 constexpr int TMEM_COLS = 512;
@@ -149,9 +156,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_attn_status, 0, code); }
 
-/* Slow path of mbar_wait. */
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
-                                            uint64_t limit_ns) {
+/* Slow path of mbar_wait (inlined into kernels that change their register
+ * budget with setmaxnreg, which cannot make calls; a call elsewhere). */
+__device__ __forceinline__ bool mbar_wait_slow_body(uint32_t bar, uint32_t parity,
+                                                    volatile uint32_t* abort_flag, uint64_t limit_ns) {
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 0; it < WAIT_MAX_ITERS; ++it) {
         if (mbar_try(bar, parity)) return true;
@@ -165,6 +173,11 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volat
     return false;
 }
 
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                            uint64_t limit_ns) {
+    return mbar_wait_slow_body(bar, parity, abort_flag, limit_ns);
+}
+
 /* Bounded wait for the phase of parity `parity` of an mbarrier.  Returns false
  * when another warp raised the abort flag, or after the limit (then it records
  * the timeout and raises the flag itself). */
@@ -174,14 +187,25 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     return mbar_wait_slow(bar, parity, abort_flag, limit_ns);
 }
 
+/* The same, with no call (for the setmaxnreg kernel). */
+__device__ __forceinline__ bool mbar_wait_inl(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                              uint64_t limit_ns) {
+    if (mbar_try(bar, parity)) return true;
+    return mbar_wait_slow_body(bar, parity, abort_flag, limit_ns);
+}
+
 /* Bounded wait that ignores the abort flag: used on the abort path to let the
  * CTA's own copies and MMAs in flight land before it exits. */
-__device__ __noinline__ void mbar_drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+__device__ __forceinline__ void mbar_drain_wait_inl(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 0; it < WAIT_MAX_ITERS; ++it) {
         if (mbar_try(bar, parity)) return;
         if ((it & 63u) == 63u && globaltimer() - t0 > limit_ns) return;
     }
+}
+
+__device__ __noinline__ void mbar_drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    mbar_drain_wait_inl(bar, parity, limit_ns);
 }
 
 __device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint32_t dst, uint32_t bar,
@@ -637,8 +661,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-
     if (warp == LOAD_WARP) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(OTHER_REGS) : "memory");
         /* ---------------- TMA producer ---------------- */
         if (lane == 0) {
             uint32_t it = 0;          // K/V ring position (K_j and V_j each take one)
@@ -648,7 +672,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const int idx = unit_index(r);
                 if (idx >= p.n_units) break;
                 const Unit u = unit_at<CAUSAL>(idx, p);
-                if (local > 0 && !mbar_wait(bar_q_empty, (local - 1) & 1, abort_flag, wlim)) {
+                if (local > 0 && !mbar_wait_inl(bar_q_empty, (local - 1) & 1, abort_flag, wlim)) {
                     aborted = true;
                     break;
                 }
@@ -662,7 +686,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     // one ring stage holds K_j and V_j, filled and released together
                     const int s = it % NSTAGE;
                     const uint32_t use = it / NSTAGE;
-                    if (!mbar_wait(bar_kv_empty(s), (use & 1u) ^ 1u, abort_flag, wlim)) {
+                    if (!mbar_wait_inl(bar_kv_empty(s), (use & 1u) ^ 1u, abort_flag, wlim)) {
                         aborted = true;
                         break;
                     }
@@ -684,16 +708,17 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             if (aborted) {
                 /* let this CTA's copies in flight land before the CTA exits */
-                if (local > 0) mbar_drain_wait(bar_q_full, (local - 1) & 1, wlim);
+                if (local > 0) mbar_drain_wait_inl(bar_q_full, (local - 1) & 1, wlim);
                 const uint32_t n_back = it < (uint32_t)NSTAGE ? it : (uint32_t)NSTAGE;
                 for (uint32_t b = 1; b <= n_back; ++b) {
                     const uint32_t i = it - b;
-                    mbar_drain_wait(bar_kv_full(i % NSTAGE), (i / NSTAGE) & 1u, wlim);
+                    mbar_drain_wait_inl(bar_kv_full(i % NSTAGE), (i / NSTAGE) & 1u, wlim);
                 }
             }
         }
         __syncwarp();
     } else if (warp == MMA_WARP) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(OTHER_REGS) : "memory");
         /* ---------------- MMA issuer ----------------
          * Tensor-core order per K/V block j, one thread:
          *   P0_j V_j, S0_{j+1}, P1_j V_j, S1_{j+1}
@@ -728,11 +753,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const Unit u = unit_at<CAUSAL>(idx, p);
                 const int n0 = u.n[0], n1 = u.n[1];
                 const int nmax = n0 > n1 ? n0 : n1;
-                if (!mbar_wait(bar_q_full, local & 1, abort_flag, wlim)) { aborted = true; break; }
+                if (!mbar_wait_inl(bar_q_full, local & 1, abort_flag, wlim)) { aborted = true; break; }
                 // block 0: S0_0, S1_0
                 {
                     const uint32_t st = it % NSTAGE;
-                    if (!mbar_wait(bar_kv_full(st), (it / NSTAGE) & 1u, abort_flag, wlim)) { aborted = true; break; }
+                    if (!mbar_wait_inl(bar_kv_full(st), (it / NSTAGE) & 1u, abort_flag, wlim)) { aborted = true; break; }
                     const uint64_t kd = kd_base + 2 * st * SLOT_STEP;
                     if (n0 > 0) { issue_s<D, FP8>(ts0, qd0, kd, IDESC_S); mma_commit(bs0); }
                     if (n1 > 0) { issue_s<D, FP8>(ts1, qd1, kd, IDESC_S); mma_commit(bs1); }
@@ -746,26 +771,26 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const uint32_t nx = it + 1;                      // ring position of block j+1
                     const uint64_t kd = kd_base + 2 * (nx % NSTAGE) * SLOT_STEP;
                     if (j < n0) {
-                        if (!mbar_wait(bh0, pr0 & 1u, abort_flag, wlim)) { aborted = true; break; }
+                        if (!mbar_wait_inl(bh0, pr0 & 1u, abort_flag, wlim)) { aborted = true; break; }
                         tc_fence_after();
                         issue_pv<FP8>(to0, ts0, vd, IDESC_PV, acc, 0);
-                        if (!mbar_wait(bp0, pr0 & 1u, abort_flag, wlim)) { aborted = true; break; }
+                        if (!mbar_wait_inl(bp0, pr0 & 1u, abort_flag, wlim)) { aborted = true; break; }
                         ++pr0;
                         tc_fence_after();
                         issue_pv<FP8>(to0, ts0, vd, IDESC_PV, 1u, 1);
                         if (j == n0 - 1) mma_commit(bo0);
                     }
                     if (has_next &&
-                        !mbar_wait(bar_kv_full(nx % NSTAGE), (nx / NSTAGE) & 1u, abort_flag, wlim)) {
+                        !mbar_wait_inl(bar_kv_full(nx % NSTAGE), (nx / NSTAGE) & 1u, abort_flag, wlim)) {
                         aborted = true;
                         break;
                     }
                     if (j + 1 < n0) { issue_s<D, FP8>(ts0, qd0, kd, IDESC_S); mma_commit(bs0); }
                     if (j < n1) {
-                        if (!mbar_wait(bh1, pr1 & 1u, abort_flag, wlim)) { aborted = true; break; }
+                        if (!mbar_wait_inl(bh1, pr1 & 1u, abort_flag, wlim)) { aborted = true; break; }
                         tc_fence_after();
                         issue_pv<FP8>(to1, ts1, vd, IDESC_PV, acc, 0);
-                        if (!mbar_wait(bp1, pr1 & 1u, abort_flag, wlim)) { aborted = true; break; }
+                        if (!mbar_wait_inl(bp1, pr1 & 1u, abort_flag, wlim)) { aborted = true; break; }
                         ++pr1;
                         tc_fence_after();
                         issue_pv<FP8>(to1, ts1, vd, IDESC_PV, 1u, 1);
@@ -780,10 +805,14 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             /* all MMAs this thread issued have completed once this phase lands */
             mma_commit(bar_drain);
-            mbar_drain_wait(bar_drain, 0, wlim);
+            mbar_drain_wait_inl(bar_drain, 0, wlim);
         }
         __syncwarp();
+    } else if (warp >= 8) {
+        /* warps 10, 11: no role; their registers go to the softmax warps */
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(OTHER_REGS) : "memory");
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(SOFTMAX_REGS) : "memory");
         /* ---------------- softmax + epilogue, warps 0-7 ---------------- */
         const int t = warp >> 2;                 // Q tile of this warpgroup
         const int quarter = warp & 3;            // TMEM lanes [32*quarter, 32*quarter + 32)
@@ -803,14 +832,14 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             const int idx = unit_index(r);
             if (idx >= p.n_units) break;
             const Unit u = unit_at<CAUSAL>(idx, p);
-            const int n = u.n[t];
+            const int n = t ? u.n[1] : u.n[0];   // (not u.n[t]: no local-memory copy of u)
             if (n == 0) continue;
             const int row = u.pair * UNIT_ROWS + t * BLOCK_M + row_in_tile;
             float m_ref = -INFINITY;   // reference max, log2 units of scale*q.k
             float l = 0.0f;            // running sum of 2^(c*s - m_ref)
             bool ok = true;
             for (int j = 0; j < n; ++j) {
-                ok = mbar_wait(bar_s, sph & 1u, abort_flag, wlim);
+                ok = mbar_wait_inl(bar_s, sph & 1u, abort_flag, wlim);
                 ++sph;
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
@@ -918,7 +947,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                 l += sum_a + sum_b;
             }
             if (!ok) break;
-            ok = mbar_wait(bar_o, oph & 1u, abort_flag, wlim);
+            ok = mbar_wait_inl(bar_o, oph & 1u, abort_flag, wlim);
             ++oph;
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;

@@ -28,9 +28,12 @@
  *                      dV_j += P^T dO_i               (A from TMEM)
  *                      S^T of block i+1               (overwrites P^T: MMAs run in issue order)
  *                      dK_j += dS^T Q_i               (A, B from shared memory)
- *                  and the same 8 warps add the dQ partial into the fp32
- *                  accumulator with vector atomics while the tensor cores
- *                  already work on block i+1.  At the end they write dK_j, dV_j.
+ *                  (at d = 64, where dQ has columns of its own, dQ_i after S^T)
+ *                  Warps 12-15 (thread = query row) add the dQ partial into the
+ *                  fp32 accumulator with vector atomics while warps 0-7 already
+ *                  work on block i+1.  At the end warps 0-7 write dK_j, dV_j.
+ *                  Warp 8 issues the TMA loads, warp 9 the MMAs; setmaxnreg
+ *                  gives the P/dS warps the registers of the others.
  * bwd_post_kernel  dQ accumulator -> bf16.
  *
  * The dQ accumulator is tiled [BH][Q block][D/4][128 rows][4]: the four
@@ -38,10 +41,20 @@
  * beside it, so a warp's atomic covers 512 contiguous bytes.
  */
 
-constexpr int BWD_THREADS = 320;    // warps 0-7 P, dS, dQ readout, epilogue; 8 TMA; 9 MMA
+constexpr int BWD_THREADS = 512;    // warps 0-7 P, dS, epilogue; 8 TMA; 9 MMA; 12-15 dQ readout
 constexpr int BWD_COMPUTE = 256;
 constexpr int BWD_LOAD_WARP = 8;
 constexpr int BWD_MMA_WARP = 9;
+constexpr int BWD_READ_WARP0 = 12;
+constexpr int BWD_READERS = 128;
+/* Register split (setmaxnreg) of the 512 x 128 registers the launch holds:
+ * the P/dS warpgroups rise to 176, the TMA/MMA warpgroup (with the two warps
+ * that have no role) drops to 56 and the readout warpgroup to 104. */
+constexpr int BWD_COMPUTE_REGS = 176;
+constexpr int BWD_CTRL_REGS = 56;
+constexpr int BWD_READ_REGS = 104;
+static_assert(2 * 128 * BWD_COMPUTE_REGS + 128 * BWD_CTRL_REGS + 128 * BWD_READ_REGS == BWD_THREADS * 128,
+              "register split");
 
 struct BwdParams {
     __nv_bfloat16* dq;
@@ -140,6 +153,35 @@ bwd_post_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, i
     }
 }
 
+/* dQ_i partial = dS K_j: A = dS (MN-major, shared memory), B = K_j (MN-major). */
+__device__ __forceinline__ void bwd_issue_dq(uint32_t tdq, uint64_t ds_mn, uint64_t k_mn, uint32_t idesc) {
+#pragma unroll 1
+    for (int kk = 0; kk < BLOCK_M / 16; ++kk) {
+        const uint64_t off = static_cast<uint64_t>((kk * 16 * 128) >> 4);
+        mma_ss(tdq, ds_mn + off, k_mn + off, idesc, kk > 0 ? 1u : 0u);
+    }
+}
+
+/* dV_j += P^T dO_i: A = P^T (TMEM), B = dO_i (MN-major). */
+__device__ __forceinline__ void bwd_issue_dv(uint32_t tdv, uint32_t ta, uint64_t do_mn, uint32_t idesc,
+                                             bool accumulate) {
+#pragma unroll 1
+    for (int kk = 0; kk < BLOCK_M / 16; ++kk) {
+        const uint64_t off = static_cast<uint64_t>((kk * 16 * 128) >> 4);
+        mma_ts(tdv, ta + bwd_p_col(kk), do_mn + off, idesc, (accumulate || kk > 0) ? 1u : 0u);
+    }
+}
+
+/* Add one 32-column chunk of this thread's dQ partial row into the tiled
+ * accumulator (row base dst, column group 8 ch .. 8 ch + 7). */
+__device__ __forceinline__ void bwd_red_chunk(float* dst, int ch, const uint32_t* v) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+        atomicAdd(reinterpret_cast<float4*>(dst + (ch * 8 + e) * (BLOCK_M * 4)),
+                  make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                              __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])));
+}
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -176,7 +218,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(bar_dp, 1);
         mbar_init(bar_p, BWD_COMPUTE);
         mbar_init(bar_dq, 1);
-        mbar_init(bar_dqf, BWD_COMPUTE);
+        mbar_init(bar_dqf, BWD_READERS);
         mbar_init(bar_dkv, 1);
         mbar_init(bar_drain, 1);
         *abort_flag = 0u;
@@ -194,6 +236,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tmem = *tmem_slot;
 
     if (warp == BWD_LOAD_WARP) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(BWD_CTRL_REGS) : "memory");
         /* ---------------- TMA: K_j, V_j once; Q_i, dO_i per Q block ---------------- */
         if (lane == 0) {
             mbar_arrive_expect_tx(bar_kv, 2 * TILE);
@@ -204,7 +247,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             int issued = 0;
             for (int it = 0; it < nq; ++it) {
                 const int s = it & 1;
-                if (!mbar_wait(bar_empty(s), ((it >> 1) & 1) ^ 1, abort_flag, wlim)) break;
+                if (!mbar_wait_inl(bar_empty(s), ((it >> 1) & 1) ^ 1, abort_flag, wlim)) break;
                 const int ib = ib0 + it;
                 mbar_arrive_expect_tx(bar_full(s), 2 * TILE);
                 for (int c = 0; c < C::CHUNKS; ++c) {
@@ -216,15 +259,16 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 ++issued;
             }
             // every copy this thread issued lands before the CTA can exit
-            mbar_drain_wait(bar_kv, 0, wlim);
+            mbar_drain_wait_inl(bar_kv, 0, wlim);
             const int back = issued < 2 ? issued : 2;
             for (int b = 1; b <= back; ++b) {
                 const int it = issued - b;
-                mbar_drain_wait(bar_full(it & 1), (it >> 1) & 1, wlim);
+                mbar_drain_wait_inl(bar_full(it & 1), (it >> 1) & 1, wlim);
             }
         }
         __syncwarp();
     } else if (warp == BWD_MMA_WARP) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(BWD_CTRL_REGS) : "memory");
         /* ---------------- MMA issue ---------------- */
         if (lane == 0) {
             constexpr uint32_t ID_KQ = idesc_bf16_ab(BLOCK_M, BLOCK_M, false, false);  // S^T, dP^T
@@ -237,8 +281,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint64_t k_mn = sdesc_sw128(sK, CHUNK_BYTES, 1024);       // K_j as MN-major B
             const uint64_t ds_mn = sdesc_sw128(sDS, 16384, 1024);           // dS as MN-major A (dQ)
             const uint64_t ds_k = sdesc_sw128(sDS, 16, 1024);               // dS^T as K-major A (dK)
-            bool ok = mbar_wait(bar_kv, 0, abort_flag, wlim);
-            if (ok) ok = mbar_wait(bar_full(0), 0, abort_flag, wlim);
+            bool ok = mbar_wait_inl(bar_kv, 0, abort_flag, wlim);
+            if (ok) ok = mbar_wait_inl(bar_full(0), 0, abort_flag, wlim);
             if (ok) {
                 tc_fence_after();
                 issue_qk<D>(ta, kd, sdesc_sw128(base + C::Q_OFF, 16, 1024), ID_KQ);  // S^T = K Q^T
@@ -249,43 +293,43 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const uint32_t sq = base + C::Q_OFF + s * TILE, sdo = base + C::DO_OFF + s * TILE;
                 if (C::DQ_OVER_DP && it > 0) {
                     // dP^T overwrites the previous dQ partial: wait until it was read out
-                    ok = mbar_wait(bar_dqf, (it - 1) & 1, abort_flag, wlim);
+                    ok = mbar_wait_inl(bar_dqf, (it - 1) & 1, abort_flag, wlim);
                     if (!ok) break;
                     tc_fence_after();
                 }
                 issue_qk<D>(tb, vd, sdesc_sw128(sdo, 16, 1024), ID_KQ);         // dP^T = V dO^T
                 mma_commit(bar_dp);
-                ok = mbar_wait(bar_p, it & 1, abort_flag, wlim);
+                ok = mbar_wait_inl(bar_p, it & 1, abort_flag, wlim);
                 if (!ok) break;
                 tc_fence_after();
-                if (!C::DQ_OVER_DP && it > 0) {
-                    ok = mbar_wait(bar_dqf, (it - 1) & 1, abort_flag, wlim);
-                    if (!ok) break;
-                    tc_fence_after();
-                }
                 const uint64_t do_mn = sdesc_sw128(sdo, CHUNK_BYTES, 1024);
                 const uint64_t q_mn = sdesc_sw128(sq, CHUNK_BYTES, 1024);
-#pragma unroll
-                for (int kk = 0; kk < BLOCK_M / 16; ++kk) {
-                    const uint64_t off = static_cast<uint64_t>((kk * 16 * 128) >> 4);
-                    mma_ss(tdq, ds_mn + off, k_mn + off, ID_DQ, kk > 0 ? 1u : 0u);  // dQ = dS K
+                // d = 128: dQ first (its columns hold the next dP^T, so the readout
+                // gates the next block); d = 64: dV and the next S^T first
+                if (C::DQ_OVER_DP) {
+                    bwd_issue_dq(tdq, ds_mn, k_mn, ID_DQ);
+                    mma_commit(bar_dq);
                 }
-                mma_commit(bar_dq);
-#pragma unroll
-                for (int kk = 0; kk < BLOCK_M / 16; ++kk) {
-                    const uint64_t off = static_cast<uint64_t>((kk * 16 * 128) >> 4);
-                    mma_ts(tdv, ta + bwd_p_col(kk), do_mn + off, ID_ACC,
-                           (it > 0 || kk > 0) ? 1u : 0u);                         // dV += P^T dO
-                }
+                bwd_issue_dv(tdv, ta, do_mn, ID_ACC, it > 0);
                 if (it + 1 < nq) {
+                    // the next S^T over P^T: the tensor core reads P^T for dV first
                     const int s1 = s ^ 1;
-                    ok = mbar_wait(bar_full(s1), ((it + 1) >> 1) & 1, abort_flag, wlim);
+                    ok = mbar_wait_inl(bar_full(s1), ((it + 1) >> 1) & 1, abort_flag, wlim);
                     if (!ok) break;
                     tc_fence_after();
                     issue_qk<D>(ta, kd, sdesc_sw128(base + C::Q_OFF + s1 * TILE, 16, 1024), ID_KQ);
                     mma_commit(bar_s);
                 }
-#pragma unroll
+                if (!C::DQ_OVER_DP) {
+                    if (it > 0) {
+                        ok = mbar_wait_inl(bar_dqf, (it - 1) & 1, abort_flag, wlim);
+                        if (!ok) break;
+                        tc_fence_after();
+                    }
+                    bwd_issue_dq(tdq, ds_mn, k_mn, ID_DQ);
+                    mma_commit(bar_dq);
+                }
+#pragma unroll 1
                 for (int kk = 0; kk < BLOCK_M / 16; ++kk) {
                     const uint64_t off_mn = static_cast<uint64_t>((kk * 16 * 128) >> 4);
                     const uint64_t off_k = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
@@ -296,14 +340,43 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             if (ok) mma_commit(bar_dkv);
             mma_commit(bar_drain);
-            mbar_drain_wait(bar_drain, 0, wlim);
+            mbar_drain_wait_inl(bar_drain, 0, wlim);
         }
         __syncwarp();
+    } else if (warp >= BWD_READ_WARP0) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(BWD_READ_REGS) : "memory");
+        /* ---------------- warps 12-15: dQ partial (thread = query row r) into the
+         * tiled accumulator; the dQ columns are released once read, before the
+         * last atomics go out ---------------- */
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        for (int it = 0; it < nq; ++it) {
+            const int ib = ib0 + it;
+            bool ok = mbar_wait_inl(bar_dq, it & 1, abort_flag, wlim);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            float* dst = p.dq_acc + (static_cast<int64_t>(bh) * p.nblk + ib) * (BLOCK_M * D) + r * 4;
+#pragma unroll 1
+            for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t v[32];
+                tmem_ld32_wait(lane_base + C::DQ_COL + ch * 32, v);
+                if (ch == D / 32 - 1) {          // every column read: release them
+                    tc_fence_before();
+                    mbar_arrive(bar_dqf);
+                }
+                bwd_red_chunk(dst, ch, v);
+            }
+        }
+    } else if (warp >= 8) {
+        /* warps 10, 11: no role; their registers go to the P/dS warpgroups */
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(BWD_CTRL_REGS) : "memory");
     } else {
-        /* ---------------- warps 0-7: P^T, dS, dQ readout, dK/dV epilogue ----------------
-         * thread = TMEM lane: K/V row r while P and dS are formed, query row r
-         * while dQ is read out; warp w covers lanes 32 (w % 4) .. and the half
-         * h = w / 4 of the columns. */
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(BWD_COMPUTE_REGS) : "memory");
+        /* ---------------- warps 0-7: P^T, dS, dK/dV epilogue ----------------
+         * thread = TMEM lane = K/V row r; warp w covers lanes 32 (w % 4) .. and
+         * the half h = w / 4 of the queries. */
         const int quarter = warp & 3, h = warp >> 2;
         const int r = quarter * 32 + lane;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -311,7 +384,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bool ok = true;
         for (int it = 0; it < nq; ++it) {
             const int ib = ib0 + it;
-            ok = mbar_wait(bar_s, it & 1, abort_flag, wlim);
+            ok = mbar_wait_inl(bar_s, it & 1, abort_flag, wlim);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
@@ -342,7 +415,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 tmem_st16(lane_base + C::RA + 64 * h + 16 * ch, pk);
             }
-            ok = mbar_wait(bar_dp, it & 1, abort_flag, wlim);
+            ok = mbar_wait_inl(bar_dp, it & 1, abort_flag, wlim);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
@@ -380,28 +453,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // dS visible to the MMA
             mbar_arrive(bar_p);
 
-            // dQ partial (thread = query row r) into the tiled accumulator
-            ok = mbar_wait(bar_dq, it & 1, abort_flag, wlim);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            tc_fence_after();
-            float* dst = p.dq_acc + (static_cast<int64_t>(bh) * p.nblk + ib) * (BLOCK_M * D) + r * 4;
-#pragma unroll
-            for (int ch = 0; ch < D / 64; ++ch) {
-                const int c0 = h * (D / 2) + ch * 32;
-                uint32_t v[32];
-                tmem_ld32_wait(lane_base + C::DQ_COL + c0, v);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    atomicAdd(reinterpret_cast<float4*>(dst + (c0 / 4 + e) * (BLOCK_M * 4)),
-                              make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                          __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])));
-            }
-            tc_fence_before();
-            mbar_arrive(bar_dqf);
         }
         if (ok) {
-            ok = mbar_wait(bar_dkv, 0, abort_flag, wlim);
+            ok = mbar_wait_inl(bar_dkv, 0, abort_flag, wlim);
             ok = __all_sync(0xffffffffu, ok);
         }
         if (ok) {

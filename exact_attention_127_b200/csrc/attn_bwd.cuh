@@ -28,17 +28,18 @@
  *                      dV_j += P^T dO_i               (A from TMEM)
  *                      S^T of block i+1               (overwrites P^T: MMAs run in issue order)
  *                      dK_j += dS^T Q_i               (A, B from shared memory)
- *                  (at d = 64, where dQ has columns of its own, dQ_i after S^T)
- *                  Warps 12-15 (thread = query row) add the dQ partial into the
- *                  fp32 accumulator with vector atomics while warps 0-7 already
+ *                  (at d = 64, where dQ has TMEM columns of its own, dQ_i after S^T)
+ *                  Warps 12-15 (thread = query row) copy the dQ partial into the
+ *                  freed Q_i / dO_i stage, and one of them adds it into the fp32
+ *                  accumulator with TMA bulk reduce-adds, while warps 0-7 already
  *                  work on block i+1.  At the end warps 0-7 write dK_j, dV_j.
  *                  Warp 8 issues the TMA loads, warp 9 the MMAs; setmaxnreg
  *                  gives the P/dS warps the registers of the others.
  * bwd_post_kernel  dQ accumulator -> bf16.
  *
- * The dQ accumulator is tiled [BH][Q block][D/4][128 rows][4]: the four
- * columns a thread adds with one vector atomic sit next to those of the rows
- * beside it, so a warp's atomic covers 512 contiguous bytes.
+ * The dQ accumulator is tiled [BH][Q block][D/4][128 rows][4], so a Q block's
+ * partial is one contiguous 128 x D fp32 region: two bulk reduce-adds of its
+ * halves, staged in the same layout in shared memory.
  */
 
 constexpr int BWD_THREADS = 512;    // warps 0-7 P, dS, epilogue; 8 TMA; 9 MMA; 12-15 dQ readout
@@ -78,7 +79,7 @@ struct BwdCfg {
     static constexpr uint32_t DO_OFF = 4 * TILE;                // [2] stages
     static constexpr uint32_t DS_OFF = 6 * TILE;                // 128 x 128 bf16 = 32 KB
     static constexpr uint32_t BAR_OFF = DS_OFF + 32768;
-    static constexpr int NUM_BARS = 12;
+    static constexpr int NUM_BARS = 15;
     static constexpr uint32_t MISC_OFF = BAR_OFF + 8 * NUM_BARS;
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
     // TMEM columns: S^T / P^T, dP^T, the dV and dK accumulators, the dQ partial
@@ -172,14 +173,11 @@ __device__ __forceinline__ void bwd_issue_dv(uint32_t tdv, uint32_t ta, uint64_t
     }
 }
 
-/* Add one 32-column chunk of this thread's dQ partial row into the tiled
- * accumulator (row base dst, column group 8 ch .. 8 ch + 7). */
-__device__ __forceinline__ void bwd_red_chunk(float* dst, int ch, const uint32_t* v) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-        atomicAdd(reinterpret_cast<float4*>(dst + (ch * 8 + e) * (BLOCK_M * 4)),
-                  make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                              __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])));
+/* fp32 add of `bytes` bytes of shared memory at src into global memory at dst
+ * by the TMA engine (both 16-byte aligned, bytes a multiple of 16). */
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;"
+                 ::"l"(reinterpret_cast<uint64_t>(dst)), "r"(src), "r"(bytes) : "memory");
 }
 
 template <int D, bool CAUSAL>
@@ -198,8 +196,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t bar_kv = bars;
     auto bar_full = [&](int s) { return bars + 8 + 8u * s; };
     auto bar_empty = [&](int s) { return bars + 24 + 8u * s; };
-    const uint32_t bar_s = bars + 40, bar_p = bars + 48, bar_dq = bars + 56, bar_dqf = bars + 64;
+    const uint32_t bar_s = bars + 40, bar_p = bars + 48, bar_dqf = bars + 64;   // (bars + 56 unused)
     const uint32_t bar_dkv = bars + 72, bar_drain = bars + 80, bar_dp = bars + 88;
+    auto bar_free = [&](int s) { return bars + 96 + 8u * s; };   // stage s handed back by the readout
+    const uint32_t bar_rd = bars + 112;                          // the dQ tile is in shared memory
     uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::MISC_OFF);
     volatile uint32_t* const abort_flag = reinterpret_cast<volatile uint32_t*>(base_ptr + C::MISC_OFF + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -213,11 +213,12 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar_full(s), 1);
             mbar_init(bar_empty(s), 1);
+            mbar_init(bar_free(s), 1);
         }
+        mbar_init(bar_rd, BWD_READERS);
         mbar_init(bar_s, 1);
         mbar_init(bar_dp, 1);
         mbar_init(bar_p, BWD_COMPUTE);
-        mbar_init(bar_dq, 1);
         mbar_init(bar_dqf, BWD_READERS);
         mbar_init(bar_dkv, 1);
         mbar_init(bar_drain, 1);
@@ -247,7 +248,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             int issued = 0;
             for (int it = 0; it < nq; ++it) {
                 const int s = it & 1;
-                if (!mbar_wait_inl(bar_empty(s), ((it >> 1) & 1) ^ 1, abort_flag, wlim)) break;
+                if (!mbar_wait_inl(bar_free(s), ((it >> 1) & 1) ^ 1, abort_flag, wlim)) break;
                 const int ib = ib0 + it;
                 mbar_arrive_expect_tx(bar_full(s), 2 * TILE);
                 for (int c = 0; c < C::CHUNKS; ++c) {
@@ -304,12 +305,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc_fence_after();
                 const uint64_t do_mn = sdesc_sw128(sdo, CHUNK_BYTES, 1024);
                 const uint64_t q_mn = sdesc_sw128(sq, CHUNK_BYTES, 1024);
-                // d = 128: dQ first (its columns hold the next dP^T, so the readout
-                // gates the next block); d = 64: dV and the next S^T first
-                if (C::DQ_OVER_DP) {
-                    bwd_issue_dq(tdq, ds_mn, k_mn, ID_DQ);
-                    mma_commit(bar_dq);
-                }
+                // d = 128: dQ first (measured faster); d = 64, where the dQ partial
+                // has TMEM columns of its own: dV and the next S^T first
+                if (C::DQ_OVER_DP) bwd_issue_dq(tdq, ds_mn, k_mn, ID_DQ);
                 bwd_issue_dv(tdv, ta, do_mn, ID_ACC, it > 0);
                 if (it + 1 < nq) {
                     // the next S^T over P^T: the tensor core reads P^T for dV first
@@ -327,7 +325,6 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         tc_fence_after();
                     }
                     bwd_issue_dq(tdq, ds_mn, k_mn, ID_DQ);
-                    mma_commit(bar_dq);
                 }
 #pragma unroll 1
                 for (int kk = 0; kk < BLOCK_M / 16; ++kk) {
@@ -345,19 +342,25 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         __syncwarp();
     } else if (warp >= BWD_READ_WARP0) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(BWD_READ_REGS) : "memory");
-        /* ---------------- warps 12-15: dQ partial (thread = query row r) into the
-         * tiled accumulator; the dQ columns are released once read, before the
-         * last atomics go out ---------------- */
+        /* ---------------- warps 12-15: the dQ partial of Q block i ----------------
+         * Once dK_i has read Q_i (so the stage of Q_i and dO_i is free), thread
+         * r = query row copies its row of the partial from TMEM into that stage,
+         * laid out as the accumulator tile (first half over Q_i, second over
+         * dO_i), and releases the dQ columns.  One thread then adds the tile into
+         * the fp32 accumulator with two TMA bulk reduce-adds and hands the stage
+         * back to the producer once they have read it: no atomics through the
+         * SM's load/store path. */
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const bool leader = threadIdx.x == BWD_READ_WARP0 * 32;
         for (int it = 0; it < nq; ++it) {
-            const int ib = ib0 + it;
-            bool ok = mbar_wait_inl(bar_dq, it & 1, abort_flag, wlim);
+            const int s = it & 1, ib = ib0 + it;
+            bool ok = mbar_wait_inl(bar_empty(s), (it >> 1) & 1, abort_flag, wlim);   // dK_i done
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            float* dst = p.dq_acc + (static_cast<int64_t>(bh) * p.nblk + ib) * (BLOCK_M * D) + r * 4;
+            const uint32_t sq = base + C::Q_OFF + s * TILE, sdo = base + C::DO_OFF + s * TILE;
 #pragma unroll 1
             for (int ch = 0; ch < D / 32; ++ch) {
                 uint32_t v[32];
@@ -366,9 +369,27 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tc_fence_before();
                     mbar_arrive(bar_dqf);
                 }
-                bwd_red_chunk(dst, ch, v);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int g = ch * 8 + e;     // float4 column group of the tile
+                    const uint32_t dst = (g < D / 8 ? sq : sdo) + ((g % (D / 8)) * BLOCK_M + r) * 16;
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[4 * e]),
+                                 "r"(v[4 * e + 1]), "r"(v[4 * e + 2]), "r"(v[4 * e + 3]) : "memory");
+                }
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the TMA
+            mbar_arrive(bar_rd);
+            if (leader) {
+                if (!mbar_wait_inl(bar_rd, it & 1, abort_flag, wlim)) break;
+                float* tile = p.dq_acc + (static_cast<int64_t>(bh) * p.nblk + ib) * (BLOCK_M * D);
+                bulk_reduce_add_f32(tile, sq, TILE);
+                bulk_reduce_add_f32(tile + TILE / 4, sdo, TILE);
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // the stage is read
+                mbar_arrive(bar_free(s));
             }
         }
+        if (leader) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");   // reduces complete
     } else if (warp >= 8) {
         /* warps 10, 11: no role; their registers go to the P/dS warpgroups */
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(BWD_CTRL_REGS) : "memory");

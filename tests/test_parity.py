@@ -149,6 +149,15 @@ def test_large_logits(attn, causal):
     _full_check(attn, q, k, v, causal, label="large logits")
 
 
+@pytest.mark.parametrize("N", [1024, 1100])
+def test_large_logits_d64(attn, N):
+    """d = 64, non-causal, peaked softmax.  An even number of 128-row Q tiles
+    (N = 1024, and 1100 with a ragged tail) runs the three-S-buffer pipeline,
+    including its rescale path."""
+    q, k, v = inputs.make_qkv(1, 3, N, 64, seed=14, qk_std=4.0, v_dist="uniform")
+    _full_check(attn, q, k, v, False, label=f"large logits d64 N={N}")
+
+
 def test_increasing_scores_force_rescales(attn):
     """Scores that grow along the keys move the reference max in every block."""
     N, d = 1024, 64

@@ -7,7 +7,7 @@
  * product bound by reading the K/V cache from device memory).  The key range is
  * cut into splits that run in parallel and are merged afterwards ("Q31：
  * FlashAttention 为什么快", follow-up 3), with the merge rule of the online
- * softmax (page 2, section 5.2): partial results that share a reference max
+ * softmax ("GPU 学习日报 Day 21", section 5.2): partial results that share a reference max
  * add, others are rescaled by 2^(m_old - m_new) first.
  *
  * The work is a stream over K and V with ~1 FLOP per byte, so it runs on the

@@ -6,30 +6,33 @@
  *   O = softmax(scale * Q K^T [+ causal mask]) V  and  LSE_i = ln sum_j e^{s_ij}
  * ("GPU 学习日报 Day 21", sections 3.1 and 5.3; the saved statistic of airsota
  * "science-depth-m4-047", section 3 point (c)).  The N x N matrices S and P
- * exist only tile by tile on chip (page 2, section 4): S in tensor memory
- * (TMEM), P overwriting S in TMEM as bf16, never in device memory.
+ * exist only tile by tile on chip ("GPU 学习日报 Day 21", section 4): S in
+ * tensor memory (TMEM), P overwriting S in TMEM as bf16, never in device memory.
  *
- * How it maps onto sm_100a (one persistent CTA per SM, 10 warps):
+ * How it maps onto sm_100a (one persistent CTA per SM, 12 warps in three
+ * warpgroups; setmaxnreg gives the two softmax warpgroups 208 registers per
+ * thread and the third, which holds the TMA and MMA warps, 88):
  *   warp 8      TMA producer: Q tiles once per work unit, then K_j, V_j through
  *               a ring of shared-memory stages guarded by mbarriers.
  *   warp 9      MMA issuer (one thread): tcgen05.mma S_t = Q_t K_j^T into TMEM
  *               (both operands in shared memory), then O_t += P_t V_j with P_t
  *               read from TMEM and V_j from shared memory.  It also owns the
  *               TMEM allocation (512 columns).
+ *   warps 10-11 no role (they complete the third warpgroup).
  *   warps 0-3   softmax for Q tile 0; warps 4-7 softmax for Q tile 1.  Thread
  *               r owns row r of its tile, which is TMEM lane r, so the row max
- *               and row sum need no shuffles.  Online recurrence of page 2,
- *               section 5.3, in base 2 with log2(e) folded into the scale,
+ *               and row sum need no shuffles.  Online recurrence of "GPU 学习日报
+ *               Day 21", section 5.3, in base 2 with log2(e) folded into the scale,
  *               with lazy rescaling: the reference max only moves when a block
  *               max exceeds it by more than TAU (so e^{s-m} <= 2^TAU), which is
  *               exact because numerator and denominator share the reference
- *               (page 2, section 5.2).  At the end of a unit the same warps
+ *               (the same page, section 5.2).  At the end of a unit the same warps
  *               divide O by l, round to bf16 and store O and LSE.
  *   A work unit is a pair of 128-row Q tiles of one head; the two tiles share
  *   every K/V block and ping-pong on the tensor core (while one tile's softmax
  *   runs, the other tile's GEMMs run).  Causal: blocks above the diagonal are
  *   never loaded or computed; only the diagonal block is masked element-wise
- *   (page 2, section 6 table).  Units are ordered longest first and dealt to
+ *   (the same page, section 6 table).  Units are ordered longest first and dealt to
  *   the persistent CTAs in snake order.
  *
  * Every wait on an mbarrier is bounded (iterations and wall time); when one

@@ -10,7 +10,7 @@
  *   statistic the backward pass recomputes from (airsota "science-depth-m4-047",
  *   section 3, point (c)), read as the natural-log log-sum-exp
  *       LSE_i = ln( sum_{j allowed} exp(scale * q_i . k_j) ).
- *   The result is computed as in sections 4-5 of page 2: one fused kernel that
+ *   The result is computed as in sections 4-5 of "GPU 学习日报 Day 21": one fused kernel that
  *   tiles Q, K and V through on-chip memory with the online-softmax recurrence,
  *   so the N x N score and probability matrices never reach device memory.
  *

@@ -20,7 +20,7 @@ marshals arrays.  Sources of each definition (FlashAttention teaching pages):
   5.1/5.2 and practice exercise 2 (online vs two-pass).
 * ``prob_row`` -- the probability row P_i of ``attention_rows``.
 * ``attention_qk`` -- the same definition for Nq query rows against Nk keys
-  (non-causal; the decode case Nq = 1 of page 2, section 9 and FAQ Q5).
+  (non-causal; the decode case Nq = 1 of "GPU 学习日报 Day 21", section 9 and FAQ Q5).
 * ``attention_backward`` -- gradients of sum(dO * O) with respect to q, k, v:
   the chain rule through the three steps, every N x N matrix materialised
   (the gradients the backward pass recomputes from saved statistics,

@@ -16,15 +16,15 @@
  *   - The saved statistic for the backward pass (airsota "science-depth-m4-047",
  *     section 3, point (c)) is read as the natural-log log-sum-exp of the scaled,
  *     masked score row:  LSE_i = m_i + ln(sum_j e^{s_ij - m_i}).
- *   - Same page 2, sections 5.2 and 5.3: the one-pass online recurrence
+ *   - "GPU 学习日报 Day 21", sections 5.2 and 5.3: the one-pass online recurrence
  *         m_new = max(m_old, m_block)
  *         l_new = e^{m_old - m_new} l_old + sum_block e^{x - m_new}
  *         O_acc = e^{m_old - m_new} O_acc + e^{S_block - m_new} V_block
  *         O     = O_acc / l   (once, after the last block)
  *     is provided as a second, independent function so that the tests can pin
  *     the two against each other (the pages claim exact equality up to
- *     floating-point order: page 2 FAQ Q1; page 1 section 3).
- *   - The backward pass (page 1, section 3, point (c): gradients recomputed
+ *     floating-point order: "GPU 学习日报 Day 21" FAQ Q1; "science-depth-m4-047" section 3).
+ *   - The backward pass ("science-depth-m4-047", section 3, point (c): gradients recomputed
  *     from the saved statistics) is checked against the gradients of the same
  *     definition, written out in fp64 with every N x N matrix materialised:
  *         dV = P^T dO,  dP = dO V^T,  dS_ij = P_ij (dP_ij - sum_k P_ik dP_ik),
@@ -45,7 +45,7 @@
 #include <string.h>
 
 /* ------------------------------------------------------------------------ */
-/* Softmax of one vector, two passes (page 2, section 5.1).                  */
+/* Softmax of one vector, two passes ("GPU 学习日报 Day 21", section 5.1).                  */
 /* ------------------------------------------------------------------------ */
 int oracle_softmax_two_pass(const double* x, int64_t n, double* p) {
     if (n <= 0 || !x || !p) return -1;
@@ -59,7 +59,7 @@ int oracle_softmax_two_pass(const double* x, int64_t n, double* p) {
 
 /*
  * Softmax of one vector with the online recurrence, block by block
- * (page 2, section 5.2 and its practice exercise 2).  After block b the
+ * ("GPU 学习日报 Day 21", section 5.2 and its practice exercise 2).  After block b the
  * statistics (m, l) describe x[0 .. end of block b]; the outputs written so far
  * are rescaled by the correction factor e^{m_old - m_new}.  The correction
  * factor of every block is written to factors[b] when factors is non-null
@@ -132,7 +132,7 @@ static void attention_row_three_step(const double* qi, const double* K, const do
 
 /*
  * One row of the online (FlashAttention) recurrence with key blocks of size
- * `block` (page 2, section 5.3).  Every key block: scores, block max,
+ * `block` ("GPU 学习日报 Day 21", section 5.3).  Every key block: scores, block max,
  * correction factor, rescale of l and O_acc, accumulate e^{s - m_new} V.
  * Normalise once at the end.
  */
@@ -252,8 +252,8 @@ int oracle_attention_rows(const double* q, const double* k, const double* v, int
 
 /*
  * Non-causal attention of Nq query rows against Nk key/value rows per head
- * (the decode case, Nq = 1: one new query attends to every cached key; page 2,
- * section 9 and FAQ Q5).  q: [BH, Nq, d]; k, v: [BH, Nk, d].  The same
+ * (the decode case, Nq = 1: one new query attends to every cached key;
+ * "GPU 学习日报 Day 21", section 9 and FAQ Q5).  q: [BH, Nq, d]; k, v: [BH, Nk, d].  The same
  * three-step definition per row.
  */
 int oracle_attention_rows_qk(const double* q, const double* k, const double* v, int64_t BH,

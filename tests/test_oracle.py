@@ -155,7 +155,7 @@ def test_key_value_permutation_invariance_noncausal():
 def test_key_shift_moves_lse_not_output(causal):
     """Adding c to every key row shifts row i's scores by scale*q_i.c: O is
     unchanged, LSE_i moves by exactly that amount (the invariance the online
-    recurrence rests on, page 2 section 5.2)."""
+    recurrence rests on, "GPU 学习日报 Day 21" section 5.2)."""
     q, k, v = (_rand((1, 2, 33, 8), s) for s in (19, 20, 21))
     c = _rand(8, 22)
     scale = 0.3
@@ -367,7 +367,7 @@ def test_decode_single_key_and_zero_query():
 @pytest.mark.parametrize("split", [1, 17, 64, 99])
 def test_split_and_merge_matches_whole(split):
     """Q31, follow-up 3 (split K/V, compute the parts, merge) with the merge
-    rule of the online recurrence (page 2, section 5.2): weights e^{LSE_part}."""
+    rule of the online recurrence ("GPU 学习日报 Day 21", section 5.2): weights e^{LSE_part}."""
     N = 100
     q = _rand((1, 2, 1, 16), 68, 2.0)
     k, v = _rand((1, 2, N, 16), 69, 2.0), _rand((1, 2, N, 16), 70)

@@ -248,6 +248,25 @@ int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
         workspace_bytes < decode_ws_bytes(BH, N, d))
         return ATTN_ERR_WORKSPACE;
+    {
+        // outputs (o, lse, the workspace) may not overlap the inputs or each other
+        const uintptr_t qb0 = reinterpret_cast<uintptr_t>(q), kb0 = reinterpret_cast<uintptr_t>(k);
+        const uintptr_t vb0 = reinterpret_cast<uintptr_t>(v);
+        const uintptr_t out0[3] = {reinterpret_cast<uintptr_t>(o), reinterpret_cast<uintptr_t>(lse),
+                                   reinterpret_cast<uintptr_t>(workspace)};
+        const size_t outn[3] = {static_cast<size_t>(BH * d) * 2, static_cast<size_t>(BH) * 4,
+                                decode_ws_bytes(BH, N, d)};
+        const uintptr_t in0[3] = {qb0, kb0, vb0};
+        const size_t inn[3] = {static_cast<size_t>(BH * d) * 2, static_cast<size_t>(BH * N * d) * 2,
+                               static_cast<size_t>(BH * N * d) * 2};
+        auto overlap = [](uintptr_t a, size_t na, uintptr_t b, size_t nb) { return a < b + nb && b < a + na; };
+        for (int a = 0; a < 3; ++a) {
+            for (int b = 0; b < 3; ++b)
+                if (overlap(out0[a], outn[a], in0[b], inn[b])) return ATTN_ERR_OVERLAP;
+            for (int b = a + 1; b < 3; ++b)
+                if (overlap(out0[a], outn[a], out0[b], outn[b])) return ATTN_ERR_OVERLAP;
+        }
+    }
     int dev = 0, major = 0, minor = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||

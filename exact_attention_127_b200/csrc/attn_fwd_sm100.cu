@@ -1304,6 +1304,19 @@ int fp8_impl(const void* q, const void* k, const void* v, float q_descale, float
  * pass follow. */
 #include "attn_standard.cuh"
 
+/* ATTN_ERR_OVERLAP when an output range (a device workspace counts as one)
+ * overlaps an input range or another output range; checked before any launch. */
+int check_overlaps(const void* const* outs, const size_t* out_bytes, int n_out,
+                   const void* const* ins, const size_t* in_bytes, int n_in) {
+    for (int a = 0; a < n_out; ++a) {
+        for (int b = 0; b < n_in; ++b)
+            if (ranges_overlap(outs[a], out_bytes[a], ins[b], in_bytes[b])) return ATTN_ERR_OVERLAP;
+        for (int b = a + 1; b < n_out; ++b)
+            if (ranges_overlap(outs[a], out_bytes[a], outs[b], out_bytes[b])) return ATTN_ERR_OVERLAP;
+    }
+    return ATTN_OK;
+}
+
 /* The unfused three-kernel path (S and P through device memory), host side. */
 size_t std_ws_bytes(int64_t BH, int64_t N) {
     const int64_t Np = (N + BLOCK_M - 1) / BLOCK_M * BLOCK_M;
@@ -1379,6 +1392,14 @@ int std_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
         workspace_bytes < std_ws_bytes(BH, N))
         return ATTN_ERR_WORKSPACE;
+    {
+        const size_t tb = static_cast<size_t>(BH * N * d) * 2, lb = static_cast<size_t>(BH * N) * 4;
+        const void* outs[3] = {o, lse, workspace};
+        const size_t ob[3] = {tb, lb, std_ws_bytes(BH, N)};
+        const void* ins[3] = {q, k, v};
+        const size_t ib[3] = {tb, tb, tb};
+        if ((st = check_overlaps(outs, ob, 3, ins, ib, 3)) != ATTN_OK) return st;
+    }
     int dev = 0;
     DeviceInfo* di = nullptr;
     if ((st = device_info(&dev, &di)) != ATTN_OK) return st;
@@ -1449,6 +1470,14 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
         workspace_bytes < bwd_ws_bytes(BH, N, d))
         return ATTN_ERR_WORKSPACE;
+    {
+        const size_t tb = static_cast<size_t>(BH * N * d) * 2, lb = static_cast<size_t>(BH * N) * 4;
+        const void* outs[4] = {dq, dk, dv, workspace};
+        const size_t ob[4] = {tb, tb, tb, bwd_ws_bytes(BH, N, d)};
+        const void* ins[6] = {q, k, v, o, dout, lse};
+        const size_t ib[6] = {tb, tb, tb, tb, tb, lb};
+        if ((st = check_overlaps(outs, ob, 4, ins, ib, 6)) != ATTN_OK) return st;
+    }
     int dev = 0;
     DeviceInfo* di = nullptr;
     if ((st = device_info(&dev, &di)) != ATTN_OK) return st;

@@ -123,7 +123,8 @@ size_t attn_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
  *                      caller-owned, contents ignored on entry; calls that
  *                      overlap on the GPU must not share it.
  * A memset and three kernels are enqueued on `stream`.  Same d, scale, alignment and error
- * conventions as attn_fwd; additionally B*H <= 65535.
+ * conventions as attn_fwd; additionally B*H <= 65535, and ATTN_ERR_OVERLAP when dq, dk, dv
+ * or the workspace overlap an input or one another.
  */
 int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
              const float* lse, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N,
@@ -145,7 +146,8 @@ size_t attn_standard_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d)
  * softmax that writes P (bf16, in place) and LSE, and O = P V.  Same layouts,
  * outputs and error codes as attn_fwd, plus: N <= 32768, B*H <= 65535, and a
  * device workspace of at least attn_standard_workspace_bytes (256-byte
- * aligned, caller-owned, contents ignored on entry).
+ * aligned, caller-owned, contents ignored on entry, not overlapping the
+ * inputs or outputs: ATTN_ERR_OVERLAP).
  */
 int attn_standard(const void* q, const void* k, const void* v, void* o, float* lse,
                   int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
@@ -202,7 +204,8 @@ size_t attn_decode_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
  *         ignored.  Calls that overlap on the GPU must not share it.
  * Two kernels are enqueued on `stream` (split, then combine).  Same d, scale,
  * alignment and error conventions as attn_fwd; ATTN_ERR_WORKSPACE when the
- * workspace is missing, misaligned or too small.
+ * workspace is missing, misaligned or too small; ATTN_ERR_OVERLAP when o, lse
+ * or the workspace overlap an input or one another.
  */
 int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse,
                 int64_t B, int64_t H, int64_t N, int64_t d, float scale,

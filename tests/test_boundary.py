@@ -72,6 +72,24 @@ def test_rejects_overlapping_outputs(lib):
     assert _call(lib, lse=FAKE + 0x300000 + 64) == OVERLAP  # lse inside o
 
 
+def test_other_entry_points_reject_overlaps(lib):
+    """attn_bwd, attn_standard and attn_decode check overlaps before any launch."""
+    big = 1 << 40
+    ws = FAKE + 0x10000000                      # 256-byte aligned, far from the tensors
+    a = [FAKE + 0x100000 * i for i in range(9)]  # q k v o dout lse dq dk dv
+    assert lib.attn_bwd(*a, 1, 1, 128, 64, 0, 0.1, ws, big, None) != OVERLAP
+    b = list(a)
+    b[6] = a[0]                                  # dq on top of q
+    assert lib.attn_bwd(*b, 1, 1, 128, 64, 0, 0.1, ws, big, None) == OVERLAP
+    b = list(a)
+    b[8] = a[7] + 64                             # dv inside dk
+    assert lib.attn_bwd(*b, 1, 1, 128, 64, 0, 0.1, ws, big, None) == OVERLAP
+    assert lib.attn_bwd(*a, 1, 1, 128, 64, 0, 0.1, a[3], big, None) == OVERLAP   # workspace on o
+    assert lib.attn_standard(a[0], a[1], a[2], a[1], a[4], 1, 1, 128, 64, 0, 0.1, ws, big, None) == OVERLAP
+    assert lib.attn_decode(a[0], a[1], a[2], a[2] + 32, a[4], 1, 1, 128, 64, 0.1, ws, big, None) == OVERLAP
+    assert lib.attn_decode(a[0], a[1], a[2], a[3], a[4], 1, 1, 128, 64, 0.1, a[1], big, None) == OVERLAP
+
+
 def test_empty_problem_is_ok_without_pointers(lib):
     assert _call(lib, q=None, k=None, v=None, o=None, lse=None, B=0) == OK
     assert _call(lib, q=None, k=None, v=None, o=None, lse=None, N=0) == OK

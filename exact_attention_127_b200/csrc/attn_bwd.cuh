@@ -51,10 +51,12 @@ constexpr int BWD_READERS = 128;
 /* Register split (setmaxnreg) of the 512 x 128 registers the launch holds:
  * the P/dS warpgroups rise to 176, the TMA/MMA warpgroup (with the two warps
  * that have no role) drops to 56 and the readout warpgroup to 104. */
+constexpr int BWD_LAUNCH_REGS = 128;  // per thread at launch (checked on the host before launching)
 constexpr int BWD_COMPUTE_REGS = 176;
 constexpr int BWD_CTRL_REGS = 56;
 constexpr int BWD_READ_REGS = 104;
-static_assert(2 * 128 * BWD_COMPUTE_REGS + 128 * BWD_CTRL_REGS + 128 * BWD_READ_REGS == BWD_THREADS * 128,
+static_assert(2 * 128 * BWD_COMPUTE_REGS + 128 * BWD_CTRL_REGS + 128 * BWD_READ_REGS ==
+                  BWD_THREADS * BWD_LAUNCH_REGS,
               "register split");
 
 struct BwdParams {

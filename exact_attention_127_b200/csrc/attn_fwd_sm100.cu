@@ -67,9 +67,10 @@ constexpr int NUM_THREADS = 384;      // 3 warpgroups: softmax tile 0, softmax t
  * thread (384 x 168 = 64512); the producer/MMA warpgroup gives back down to
  * 88 so that the two softmax warpgroups can hold 208: 2*128*208 + 128*88 =
  * 64512, exactly what the launch holds (a larger sum would wait forever). */
+constexpr int LAUNCH_REGS = 168;      // per thread at launch (checked on the host before launching)
 constexpr int SOFTMAX_REGS = 208;
 constexpr int OTHER_REGS = 88;
-static_assert(2 * 128 * SOFTMAX_REGS + 128 * OTHER_REGS == NUM_THREADS * 168, "register split");
+static_assert(2 * 128 * SOFTMAX_REGS + 128 * OTHER_REGS == NUM_THREADS * LAUNCH_REGS, "register split");
 constexpr int LOAD_WARP = 8;
 constexpr int MMA_WARP = 9;
 constexpr int TMEM_COLS = 512;
@@ -1098,8 +1099,12 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
     {
         std::lock_guard<std::mutex> lock(g_mutex);
         if (!di->smem_set[key]) {
-            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
-                cudaSuccess) {
+            // the register split adds up only with LAUNCH_REGS per thread: with
+            // fewer, setmaxnreg.inc would wait for registers that never come free
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != LAUNCH_REGS ||
+                cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
+                    cudaSuccess) {
                 cudaGetLastError();
                 return ATTN_ERR_LAUNCH;
             }
@@ -1436,7 +1441,10 @@ int bwd_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
                const float* lse, const BwdParams& prm, cudaStream_t stream) {
     auto kern = bwd_main_kernel<D, CAUSAL>;
     constexpr int SMEM = BwdCfg<D>::SMEM_BYTES;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess) {
+    // the register split adds up only with BWD_LAUNCH_REGS per thread (see attn_bwd.cuh)
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != BWD_LAUNCH_REGS ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess) {
         cudaGetLastError();
         return ATTN_ERR_LAUNCH;
     }

@@ -889,7 +889,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const float neg_m = (m_ref == -INFINITY) ? 0.0f : -m_ref;
                 const uint64_t c2 = f2pack(c, c);
                 const uint64_t nm2 = f2pack(neg_m, neg_m);
-                float sum_a = 0.0f, sum_b = 0.0f;
+                uint64_t sum2 = f2pack(0.0f, 0.0f);
 #pragma unroll
                 for (int qtr = 0; qtr < 4; ++qtr) {
                     const int half = qtr >> 1;
@@ -907,8 +907,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                             p0 = ex2(x0);
                             p1 = ex2(x1);
                         }
-                        sum_a += p0;
-                        sum_b += p1;
+                        sum2 = fadd2(sum2, f2pack(p0, p1));
                         if constexpr (FP8) {
                             pq[2 * k] = p0;
                             pq[2 * k + 1] = p1;
@@ -948,7 +947,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     mbar_arrive(bar_ph);
                     mbar_arrive(bar_p);
                 }
-                l += sum_a + sum_b;
+                {
+                    float sa, sb;
+                    f2unpack(sum2, sa, sb);
+                    l += sa + sb;
+                }
             }
             if (!ok) break;
             ok = mbar_wait_inl(bar_o, oph & 1u, abort_flag, wlim);

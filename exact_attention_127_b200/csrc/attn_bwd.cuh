@@ -175,6 +175,13 @@ __device__ __forceinline__ void bwd_issue_dv(uint32_t tdv, uint32_t ta, uint64_t
     }
 }
 
+/* Elementwise product of two f32 pairs (mul.rn.f32x2). */
+__device__ __forceinline__ uint64_t bwd_fmul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
 /* fp32 add of `bytes` bytes of shared memory at src into global memory at dst
  * by the TMA engine (both 16-byte aligned, bytes a multiple of 16). */
 __device__ __forceinline__ void bulk_reduce_add_f32(float* dst, uint32_t src, uint32_t bytes) {
@@ -404,6 +411,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int r = quarter * 32 + lane;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
         const float c = p.scale_log2, sc = p.scale;
+        const uint64_t c2 = f2pack(c, c), sc2 = f2pack(sc, sc);
         bool ok = true;
         for (int it = 0; it < nq; ++it) {
             const int ib = ib0 + it;
@@ -426,10 +434,15 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {
                     const float4 l4 = __ldg(reinterpret_cast<const float4*>(lse2 + ch * 32 + e));
-                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    // c s - lse2 on pairs (f32x2: the same rounding as scalar fmaf)
+                    float x[4];
+                    f2unpack(ffma2(f2pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2,
+                                   f2pack(-l4.x, -l4.y)), x[0], x[1]);
+                    f2unpack(ffma2(f2pack(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])), c2,
+                                   f2pack(-l4.z, -l4.w)), x[2], x[3]);
 #pragma unroll
                     for (int hh = 0; hh < 4; ++hh) {
-                        float pv = ex2(fmaf(__uint_as_float(sv[e + hh]), c, -lv[hh]));
+                        float pv = ex2(x[hh]);
                         if (ch * 32 + e + hh < mask_lim) pv = 0.0f;
                         pf[ch * 32 + e + hh] = pv;
                     }
@@ -454,11 +467,17 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {
                     const float4 d4 = __ldg(reinterpret_cast<const float4*>(dvec + ch * 32 + e));
-                    const float dvv[4] = {d4.x, d4.y, d4.z, d4.w};
+                    // scale * P (dP - D) on pairs, in the scalar order (f32x2 rounds alike)
                     float dd[4];
-#pragma unroll
-                    for (int hh = 0; hh < 4; ++hh)
-                        dd[hh] = pf[ch * 32 + e + hh] * (__uint_as_float(dpv[e + hh]) - dvv[hh]) * sc;
+                    const int j = ch * 32 + e;
+                    uint64_t t01 = fsub2(f2pack(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])),
+                                         f2pack(d4.x, d4.y));
+                    uint64_t t23 = fsub2(f2pack(__uint_as_float(dpv[e + 2]), __uint_as_float(dpv[e + 3])),
+                                         f2pack(d4.z, d4.w));
+                    t01 = bwd_fmul2(bwd_fmul2(f2pack(pf[j], pf[j + 1]), t01), sc2);
+                    t23 = bwd_fmul2(bwd_fmul2(f2pack(pf[j + 2], pf[j + 3]), t23), sc2);
+                    f2unpack(t01, dd[0], dd[1]);
+                    f2unpack(t23, dd[2], dd[3]);
                     dk[e / 2] = pack_bf16(dd[0], dd[1]);
                     dk[e / 2 + 1] = pack_bf16(dd[2], dd[3]);
                 }

@@ -83,6 +83,28 @@ def test_backward_larger_causal_two_heads():
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("d", [64, 128])
+def test_backward_non_default_scale(d):
+    """scale enters P, dQ and dK: a scale other than 1/sqrt(d) must carry through."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    q, k, v = inputs.make_qkv(1, 2, 300, d, seed=45)
+    dout = inputs.make_qkv(1, 2, 300, d, seed=46)[0]
+    _check(q, k, v, dout, True, 0.3, f"scale 0.3 d={d}")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_large_logits(causal):
+    """Peaked softmax (logit std ~16): P near 0 or 1, dS dominated by few keys."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    q, k, v = inputs.make_qkv(1, 2, 700, 128, seed=47, qk_std=4.0, v_dist="uniform")
+    dout = inputs.make_qkv(1, 2, 700, 128, seed=48)[0]
+    _check(q, k, v, dout, causal, 1 / math.sqrt(128), f"large logits causal={causal}")
+
+
+@pytest.mark.gpu
 def test_backward_headline_workload_two_heads():
     """The configuration bench.py --pass bwd times (B=4, H=16, N=8192, d=128,
     causal, the same dO), checked in full on the first and the last head."""

@@ -28,7 +28,9 @@
  *                      dV_j += P^T dO_i               (A from TMEM)
  *                      S^T of block i+1               (overwrites P^T: MMAs run in issue order)
  *                      dK_j += dS^T Q_i               (A, B from shared memory)
- *                  (at d = 64, where dQ has TMEM columns of its own, dQ_i after S^T)
+ *                  (at d = 64, where dQ has TMEM columns of its own, dV_i and the
+ *                  next S^T go as soon as P^T is in TMEM, while warps 0-7 form
+ *                  dS, and dQ_i, dK_j follow)
  *                  Warps 12-15 (thread = query row) copy the dQ partial into the
  *                  freed Q_i / dO_i stage, and one of them adds it into the fp32
  *                  accumulator with TMA bulk reduce-adds, while warps 0-7 already
@@ -89,6 +91,9 @@ struct BwdCfg {
     static constexpr uint32_t RA = 0, RB = 128, DV_COL = 256, DK_COL = 256 + D;
     static constexpr uint32_t DQ_COL = (256 + 2 * D + D <= 512) ? 256 + 2 * D : RB;
     static constexpr bool DQ_OVER_DP = DQ_COL == RB;
+    // dV_i and the next S^T as soon as P^T is in TMEM, before dS: faster where
+    // dQ has columns of its own (D = 64); at D = 128 the later order measured faster
+    static constexpr bool EARLY_NEXT_S = !DQ_OVER_DP;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
@@ -205,7 +210,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t bar_kv = bars;
     auto bar_full = [&](int s) { return bars + 8 + 8u * s; };
     auto bar_empty = [&](int s) { return bars + 24 + 8u * s; };
-    const uint32_t bar_s = bars + 40, bar_p = bars + 48, bar_dqf = bars + 64;   // (bars + 56 unused)
+    const uint32_t bar_s = bars + 40, bar_p = bars + 48, bar_pt = bars + 56, bar_dqf = bars + 64;
     const uint32_t bar_dkv = bars + 72, bar_drain = bars + 80, bar_dp = bars + 88;
     auto bar_free = [&](int s) { return bars + 96 + 8u * s; };   // stage s handed back by the readout
     const uint32_t bar_rd = bars + 112;                          // the dQ tile is in shared memory
@@ -228,6 +233,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(bar_s, 1);
         mbar_init(bar_dp, 1);
         mbar_init(bar_p, BWD_COMPUTE);
+        mbar_init(bar_pt, BWD_COMPUTE);
         mbar_init(bar_dqf, BWD_READERS);
         mbar_init(bar_dkv, 1);
         mbar_init(bar_drain, 1);
@@ -309,31 +315,44 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 issue_qk<D>(tb, vd, sdesc_sw128(sdo, 16, 1024), ID_KQ);         // dP^T = V dO^T
                 mma_commit(bar_dp);
-                ok = mbar_wait_inl(bar_p, it & 1, abort_flag, wlim);
-                if (!ok) break;
-                tc_fence_after();
                 const uint64_t do_mn = sdesc_sw128(sdo, CHUNK_BYTES, 1024);
                 const uint64_t q_mn = sdesc_sw128(sq, CHUNK_BYTES, 1024);
-                // d = 128: dQ first (measured faster); d = 64, where the dQ partial
-                // has TMEM columns of its own: dV and the next S^T first
-                if (C::DQ_OVER_DP) bwd_issue_dq(tdq, ds_mn, k_mn, ID_DQ);
-                bwd_issue_dv(tdv, ta, do_mn, ID_ACC, it > 0);
-                if (it + 1 < nq) {
-                    // the next S^T over P^T: the tensor core reads P^T for dV first
+                // the next S^T over P^T: the tensor core reads P^T for dV first
+                auto issue_next_s = [&]() -> bool {
+                    if (it + 1 >= nq) return true;
                     const int s1 = s ^ 1;
-                    ok = mbar_wait_inl(bar_full(s1), ((it + 1) >> 1) & 1, abort_flag, wlim);
-                    if (!ok) break;
+                    if (!mbar_wait_inl(bar_full(s1), ((it + 1) >> 1) & 1, abort_flag, wlim)) return false;
                     tc_fence_after();
                     issue_qk<D>(ta, kd, sdesc_sw128(base + C::Q_OFF + s1 * TILE, 16, 1024), ID_KQ);
                     mma_commit(bar_s);
-                }
-                if (!C::DQ_OVER_DP) {
+                    return true;
+                };
+                if constexpr (C::EARLY_NEXT_S) {
+                    // D = 64: dV and the next S^T while warps 0-7 still form dS
+                    ok = mbar_wait_inl(bar_pt, it & 1, abort_flag, wlim);        // P^T in TMEM
+                    if (!ok) break;
+                    tc_fence_after();
+                    bwd_issue_dv(tdv, ta, do_mn, ID_ACC, it > 0);
+                    ok = issue_next_s();
+                    if (!ok) break;
+                    ok = mbar_wait_inl(bar_p, it & 1, abort_flag, wlim);         // dS in shared memory
+                    if (!ok) break;
+                    tc_fence_after();
                     if (it > 0) {
                         ok = mbar_wait_inl(bar_dqf, (it - 1) & 1, abort_flag, wlim);
                         if (!ok) break;
                         tc_fence_after();
                     }
                     bwd_issue_dq(tdq, ds_mn, k_mn, ID_DQ);
+                } else {
+                    // D = 128: dQ (over dP^T) first, then dV and the next S^T
+                    ok = mbar_wait_inl(bar_p, it & 1, abort_flag, wlim);
+                    if (!ok) break;
+                    tc_fence_after();
+                    bwd_issue_dq(tdq, ds_mn, k_mn, ID_DQ);
+                    bwd_issue_dv(tdv, ta, do_mn, ID_ACC, it > 0);
+                    ok = issue_next_s();
+                    if (!ok) break;
                 }
 #pragma unroll 1
                 for (int kk = 0; kk < BLOCK_M / 16; ++kk) {
@@ -451,6 +470,11 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 tmem_st16(lane_base + C::RA + 64 * h + 16 * ch, pk);
             }
+            if constexpr (C::EARLY_NEXT_S) {
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar_pt);    // P^T is in TMEM: dV and the next S^T may go
+            }
             ok = mbar_wait_inl(bar_dp, it & 1, abort_flag, wlim);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
@@ -490,7 +514,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                  "r"(dk[4 * u + 3]) : "memory");
                 }
             }
-            tmem_wait_st();
+            if constexpr (!C::EARLY_NEXT_S) tmem_wait_st();   // the P^T stores
             tc_fence_before();
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // dS visible to the MMA
             mbar_arrive(bar_p);

@@ -596,7 +596,7 @@ def run_standard(args, w):
 
 
 def run_decode(args, w):
-    """One step = one attn_decode call (split kernel + combine kernel) over a
+    """One step = one attn_decode call (stream kernel + combine kernel) over a
     batch of one query row per head against N cached keys; HBM-bound."""
     import torch
     import torch.distributed as dist
@@ -662,7 +662,7 @@ def run_decode(args, w):
                          "unit": "GB/s", "frac": value / world / peaks["hbm_gbs"],
                          "traffic": load_traffic(w.name),
                          "peak_source": f"{peak_src} HBM copy (MEASURED_PEAKS.json)",
-                         "kernel": "decode_split_kernel + decode_combine_kernel (one call)",
+                         "kernel": "decode_stream_kernel + decode_combine_kernel (one call)",
                          "compulsory_bytes_per_launch": nbytes},
             "e2e": None, "gpu_launches": 2 * args.steps, "clocks": sampler.summary(),
         }

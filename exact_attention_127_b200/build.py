@@ -11,7 +11,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC = os.path.join(PKG, "csrc", "attn_fwd_sm100.cu")
-SOURCES = [SRC, os.path.join(PKG, "csrc", "attn_decode.cu")]
+SOURCES = [SRC]
 HDR = os.path.join(ROOT, "include", "attn_fwd.h")
 LIB = os.path.join(PKG, "libattn127.so")
 
@@ -32,7 +32,7 @@ def nvcc_path() -> str:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    deps = SOURCES + [os.path.join(PKG, "csrc", f) for f in ("attn_standard.cuh", "attn_bwd.cuh")]
+    deps = SOURCES + [os.path.join(PKG, "csrc", f) for f in ("attn_standard.cuh", "attn_bwd.cuh", "attn_decode.cuh")]
     deps.append(HDR)
     newest = max(os.path.getmtime(f) for f in deps)
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest:

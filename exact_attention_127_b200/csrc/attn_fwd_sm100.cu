@@ -1667,3 +1667,6 @@ const char* attn_status_str(int status) {
 const char* attn_version(void) { return ATTN_VERSION; }
 
 }  // extern "C"
+
+/* Decode with split K/V: its own kernels and entry points. */
+#include "attn_decode.cuh"

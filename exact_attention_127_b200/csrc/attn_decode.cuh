@@ -16,19 +16,21 @@
  * CUDA cores and is bound by HBM; the tensor cores would add nothing.
  *
  *   decode_stream_kernel  persistent, one CTA per SM.  The K/V cache of all
- *                         heads is cut into 128-key stages (a head has
- *                         ceil(N/128) of them) and CTA c takes the contiguous
- *                         range [c P, (c+1) P) of the B*H*ceil(N/128) stages,
- *                         so every SM streams the same number of bytes.  Warp
- *                         4 loads each stage (K and V, 128 rows) with TMA into
- *                         a shared-memory ring; warps 0-3 take 32 keys each:
- *                         lane i scores key i from its row (the 128-byte
- *                         swizzle spreads the 32 rows over all banks and q is
- *                         read as a broadcast), then the warp walks the 32 keys,
- *                         broadcasting p_i, while each lane accumulates d/32
- *                         columns of p_i v_i.  At the end of each head's part of
- *                         the range the four warps merge and write one
- *                         unnormalised partial (O, m, l) to slot head + c.
+ *                         heads is cut into stages of 32 keys per consumer warp
+ *                         (128 keys and 4 warps at d = 128, 256 keys and 8 warps
+ *                         at d = 64: 64 KB of K and V either way) and CTA c takes
+ *                         the contiguous range [c P, (c+1) P) of the B*H*sph
+ *                         stages (sph per head), so every SM streams the same
+ *                         number of bytes.  The last warp loads each stage with
+ *                         TMA into a 3-stage shared-memory ring; each consumer
+ *                         warp takes 32 keys: lane i scores key i from its row
+ *                         (the 128-byte swizzle spreads the 32 rows over all
+ *                         banks and q is read as a broadcast), then the warp
+ *                         walks the 32 keys, broadcasting p_i, while each lane
+ *                         accumulates d/32 columns of p_i v_i.  At the end of
+ *                         each head's part of the range the consumer warps
+ *                         merge and write one unnormalised partial (O, m, l) to
+ *                         slot head + c.
  *   decode_combine_kernel grid = B*H CTAs of d threads; merges the partials of
  *                         a head (CTAs c0 .. c1 of its stage range), divides by
  *                         l, rounds O to bf16 and writes LSE.
@@ -40,22 +42,27 @@
 
 namespace {
 
-constexpr int DEC_CONSUMERS = 4;                        // warps 0-3 consume, warp 4 loads
-constexpr int DEC_THREADS = (DEC_CONSUMERS + 1) * 32;
-constexpr int DEC_STAGE_KEYS = 32 * DEC_CONSUMERS;      // 128 keys per stage, one per consumer lane
 constexpr int DEC_MAX_CTAS = 160;                       // >= the SMs of an sm_100 part; sizes the workspace
-constexpr uint32_t DEC_BOX_BYTES = DEC_STAGE_KEYS * 128;   // one 64-column TMA box: 128 rows x 128 B
-static_assert(DEC_STAGE_KEYS == BLOCK_M, "a stage is one box of the tensor maps encode_map makes");
+constexpr int DEC_BOX_ROWS = BLOCK_M;                   // rows of a box of the tensor maps encode_map makes
+constexpr uint32_t DEC_BOX_BYTES = DEC_BOX_ROWS * 128;  // one box: 128 rows x 64 columns x 2 B
 
+/* d = 128: 4 consumer warps, 128-key stages (two 64-column boxes per row);
+ * d = 64: 8 consumer warps, 256-key stages (two 128-row boxes), so that a stage
+ * is 64 KB either way and a warp's share of the per-key work stays the same. */
 template <int D>
 struct DecCfg {
-    static constexpr int BOXES = D / 64;                 // 64-column boxes per row
-    static constexpr uint32_t KV_BYTES = BOXES * DEC_BOX_BYTES;   // K (or V) of one stage
+    static constexpr int CONSUMERS = D == 64 ? 8 : 4;    // warps 0 .. CONSUMERS-1; the next one loads
+    static constexpr int THREADS = (CONSUMERS + 1) * 32;
+    static constexpr int STAGE_KEYS = 32 * CONSUMERS;    // one key per consumer lane
+    static constexpr int ROW_BOXES = STAGE_KEYS / DEC_BOX_ROWS;
+    static constexpr int COL_BOXES = D / 64;
+    static constexpr uint32_t COL_BOX_STRIDE = STAGE_KEYS * 128;   // bytes between 64-column boxes
+    static constexpr uint32_t KV_BYTES = COL_BOXES * COL_BOX_STRIDE;   // K (or V) of one stage
     static constexpr uint32_t STAGE_BYTES = 2 * KV_BYTES;
-    static constexpr int NSTAGE = (192 * 1024) / STAGE_BYTES;    // 3 at d = 128, 6 at d = 64
+    static constexpr int NSTAGE = (192 * 1024) / STAGE_BYTES;    // 3
     static constexpr uint32_t Q_OFF = NSTAGE * STAGE_BYTES;      // q * scale * log2(e), fp32
     static constexpr uint32_t RED_OFF = Q_OFF + D * 4;           // per warp: O row, then m, l
-    static constexpr uint32_t RED_BYTES = DEC_CONSUMERS * (D + 2) * 4;
+    static constexpr uint32_t RED_BYTES = CONSUMERS * (D + 2) * 4;
     static constexpr uint32_t BAR_OFF = (RED_OFF + RED_BYTES + 7u) & ~7u;
     static constexpr uint32_t FLAG_OFF = BAR_OFF + 16 * NSTAGE;  // full[NSTAGE], empty[NSTAGE]
     static constexpr int SMEM_BYTES = FLAG_OFF + 16 + 1024;      // + slack for the 1 KB alignment
@@ -71,19 +78,21 @@ __device__ __forceinline__ float dec_ex2(float x) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-/* Named barrier over the four consumer warps (the loader never joins it). */
+/* Named barrier over the consumer warps (the loader never joins it). */
+template <int THREADS>
 __device__ __forceinline__ void dec_consumers_sync() {
-    asm volatile("bar.sync 1, %0;" ::"n"(DEC_CONSUMERS * 32) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(THREADS) : "memory");
 }
 
 template <int D>
-__global__ void __launch_bounds__(DEC_THREADS, 1)
+__global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
 decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const __nv_bfloat16* __restrict__ q, float* __restrict__ part_o,
                      float2* __restrict__ part_ml, int N, int sph, int per_cta, int total,
                      float scale_log2, uint64_t wlim) {
     using C = DecCfg<D>;
     constexpr int CPL = D / 32;                  // output columns per lane
+    constexpr int NCW = C::CONSUMERS;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;        // the swizzle wants 1 KB alignment
@@ -99,7 +108,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::NSTAGE; ++s) {
             mbar_init(bar_full(s), 1);
-            mbar_init(bar_empty(s), DEC_CONSUMERS);      // lane 0 of each consumer warp
+            mbar_init(bar_empty(s), NCW);                // lane 0 of each consumer warp
         }
         *abort_flag = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -107,7 +116,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
     }
     __syncthreads();
 
-    if (warp == DEC_CONSUMERS) {
+    if (warp == NCW) {
         /* ---------------- loader: stage g = (head g / sph, keys 128 (g % sph) ..) ---------------- */
         if (lane == 0) {
             prefetch_tmap(&tm_k);
@@ -118,15 +127,18 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                 if (it >= C::NSTAGE &&
                     !mbar_wait(bar_empty(s), ((it / C::NSTAGE) - 1) & 1, abort_flag, wlim))
                     break;
-                const int bh = g / sph, key0 = (g - bh * sph) * DEC_STAGE_KEYS;
+                const int bh = g / sph, key0 = (g - bh * sph) * C::STAGE_KEYS;
                 const uint32_t dst = base + s * C::STAGE_BYTES;
                 mbar_arrive_expect_tx(bar_full(s), C::STAGE_BYTES);
 #pragma unroll
-                for (int b = 0; b < C::BOXES; ++b)
-                    tma_load_3d(&tm_k, dst + b * DEC_BOX_BYTES, bar_full(s), 64 * b, key0, bh);
+                for (int b = 0; b < C::COL_BOXES; ++b)
 #pragma unroll
-                for (int b = 0; b < C::BOXES; ++b)
-                    tma_load_3d(&tm_v, dst + C::KV_BYTES + b * DEC_BOX_BYTES, bar_full(s), 64 * b, key0, bh);
+                    for (int rb = 0; rb < C::ROW_BOXES; ++rb) {
+                        const uint32_t off = b * C::COL_BOX_STRIDE + rb * DEC_BOX_BYTES;
+                        tma_load_3d(&tm_k, dst + off, bar_full(s), 64 * b, key0 + rb * DEC_BOX_ROWS, bh);
+                        tma_load_3d(&tm_v, dst + C::KV_BYTES + off, bar_full(s), 64 * b,
+                                    key0 + rb * DEC_BOX_ROWS, bh);
+                    }
             }
             // the copies in flight land before the CTA may exit (after an abort too)
             for (int j = max(0, it - C::NSTAGE); j < it; ++j)
@@ -135,11 +147,11 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
         return;
     }
 
-    /* ---------------- warps 0-3: 32 keys of every stage each ---------------- */
+    /* ---------------- consumer warps: 32 keys of every stage each ---------------- */
     float* const q_s = reinterpret_cast<float*>(bp + C::Q_OFF);
-    float* const red_o = reinterpret_cast<float*>(bp + C::RED_OFF);      // [4][D]
-    float* const red_m = red_o + DEC_CONSUMERS * D;                      // [4]
-    float* const red_l = red_m + DEC_CONSUMERS;                          // [4]
+    float* const red_o = reinterpret_cast<float*>(bp + C::RED_OFF);      // [NCW][D]
+    float* const red_m = red_o + NCW * D;                                // [NCW]
+    float* const red_l = red_m + NCW;                                    // [NCW]
     const int r = 32 * warp + lane;              // this lane's key row within a stage
     bool ok = true;
     float m_w = -INFINITY;                       // warp-uniform reference max (log2 units)
@@ -152,10 +164,10 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
         const int bh = g / sph, sidx = g - bh * sph;
         if (g == lo || sidx == 0) {
             // a new head: the previous one is merged and done with q_s
-            dec_consumers_sync();
-            for (int c = threadIdx.x; c < D; c += DEC_CONSUMERS * 32)
+            dec_consumers_sync<NCW * 32>();
+            for (int c = threadIdx.x; c < D; c += NCW * 32)
                 q_s[c] = __bfloat162float(q[static_cast<int64_t>(bh) * D + c]) * scale_log2;
-            dec_consumers_sync();
+            dec_consumers_sync<NCW * 32>();
             m_w = -INFINITY;
             l_lane = 0.0f;
 #pragma unroll
@@ -164,7 +176,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
         const int s = it % C::NSTAGE;
         if (ok) ok = mbar_wait(bar_full(s), (it / C::NSTAGE) & 1, abort_flag, wlim);
         ok = __all_sync(0xffffffffu, ok);
-        const int nvalid = min(32, N - (sidx * DEC_STAGE_KEYS + 32 * warp));   // keys of this warp
+        const int nvalid = min(32, N - (sidx * C::STAGE_KEYS + 32 * warp));   // keys of this warp
         if (ok && nvalid > 0) {
             const uint8_t* kst = bp + s * C::STAGE_BYTES;
             const uint8_t* vst = kst + C::KV_BYTES;
@@ -174,7 +186,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
 #pragma unroll
             for (int u = 0; u < D / 8; ++u) {
                 const uint4 w = *reinterpret_cast<const uint4*>(
-                    kst + (u >> 3) * DEC_BOX_BYTES + r * 128 + (((u & 7) ^ (r & 7)) << 4));
+                    kst + (u >> 3) * C::COL_BOX_STRIDE + r * 128 + (((u & 7) ^ (r & 7)) << 4));
                 const float4 qa = *reinterpret_cast<const float4*>(q_s + 8 * u);
                 const float4 qb = *reinterpret_cast<const float4*>(q_s + 8 * u + 4);
                 a[0] = fmaf(bf16_lo(w.x), qa.x, a[0]);
@@ -206,7 +218,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                 const int rv = 32 * warp + i;
                 if (CPL == 4) {
                     const uint2 w = *reinterpret_cast<const uint2*>(
-                        vst + (lane >> 4) * DEC_BOX_BYTES + rv * 128 +
+                        vst + (lane >> 4) * C::COL_BOX_STRIDE + rv * 128 +
                         ((((lane & 15) >> 1) ^ (rv & 7)) << 4) + (lane & 1) * 8);
                     acc[0] = fmaf(pi, bf16_lo(w.x), acc[0]);
                     acc[1] = fmaf(pi, bf16_hi(w.x), acc[1]);
@@ -233,22 +245,22 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                 red_m[warp] = m_w;
                 red_l[warp] = l_w;
             }
-            dec_consumers_sync();
+            dec_consumers_sync<NCW * 32>();
             float M = -INFINITY;
 #pragma unroll
-            for (int w = 0; w < DEC_CONSUMERS; ++w) M = fmaxf(M, red_m[w]);
+            for (int w = 0; w < NCW; ++w) M = fmaxf(M, red_m[w]);
             const int64_t slot = static_cast<int64_t>(bh) + blockIdx.x;
-            for (int c = threadIdx.x; c < D; c += DEC_CONSUMERS * 32) {
+            for (int c = threadIdx.x; c < D; c += NCW * 32) {
                 float o = 0.0f;
 #pragma unroll
-                for (int w = 0; w < DEC_CONSUMERS; ++w)
+                for (int w = 0; w < NCW; ++w)
                     if (red_m[w] != -INFINITY) o += red_o[w * D + c] * dec_ex2(red_m[w] - M);
                 part_o[slot * D + c] = o;
             }
             if (threadIdx.x == 0) {
                 float Lsum = 0.0f;
 #pragma unroll
-                for (int w = 0; w < DEC_CONSUMERS; ++w)
+                for (int w = 0; w < NCW; ++w)
                     if (red_m[w] != -INFINITY) Lsum += red_l[w] * dec_ex2(red_m[w] - M);
                 part_ml[slot] = make_float2(M, Lsum);
             }
@@ -288,9 +300,9 @@ struct DecodePlan {
     int ctas;      // G = ceil(total / P) <= min(SMs, DEC_MAX_CTAS)
 };
 
-DecodePlan decode_plan(int64_t BH, int64_t N, int num_sms) {
+DecodePlan decode_plan(int64_t BH, int64_t N, int stage_keys, int num_sms) {
     DecodePlan pl;
-    pl.sph = static_cast<int>((N + DEC_STAGE_KEYS - 1) / DEC_STAGE_KEYS);
+    pl.sph = static_cast<int>((N + stage_keys - 1) / stage_keys);
     pl.total = static_cast<int>(BH * pl.sph);
     int64_t g0 = std::min<int64_t>(std::min(num_sms, DEC_MAX_CTAS), pl.total);
     if (g0 < 1) g0 = 1;
@@ -307,7 +319,7 @@ int decode_validate(int64_t B, int64_t H, int64_t N, int64_t d, float scale, boo
     if (*empty) return ATTN_OK;
     if (N > INT32_MAX / 2 || H > INT32_MAX / B) return ATTN_ERR_SHAPE;
     const int64_t BH = B * H;
-    const int64_t sph = (N + DEC_STAGE_KEYS - 1) / DEC_STAGE_KEYS;
+    const int64_t sph = (N + DEC_BOX_ROWS - 1) / DEC_BOX_ROWS;          // the most stages a head can have
     if (BH > (INT32_MAX - DEC_MAX_CTAS) / sph) return ATTN_ERR_SHAPE;   // stage and slot indices fit int32
     return ATTN_OK;
 }
@@ -339,7 +351,7 @@ int decode_launch(const CUtensorMap& mk, const CUtensorMap& mv, const __nv_bfloa
             set = true;
         }
     }
-    kern<<<pl.ctas, DEC_THREADS, SMEM, s>>>(mk, mv, q, part_o, part_ml, N, pl.sph, pl.per_cta,
+    kern<<<pl.ctas, DecCfg<D>::THREADS, SMEM, s>>>(mk, mv, q, part_o, part_ml, N, pl.sph, pl.per_cta,
                                             pl.total, scale_log2, WAIT_LIMIT_NS);
     decode_combine_kernel<D><<<static_cast<unsigned>(BH), D, 0, s>>>(part_o, part_ml, o, lse, pl.sph,
                                                                     pl.per_cta);
@@ -392,7 +404,8 @@ int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse
     if ((st = encode_map(enc, &mk, k, BH, N, d)) != ATTN_OK) return st;
     if ((st = encode_map(enc, &mv, v, BH, N, d)) != ATTN_OK) return st;
 
-    const DecodePlan pl = decode_plan(BH, N, di->num_sms);
+    const DecodePlan pl = decode_plan(BH, N, d == 64 ? DecCfg<64>::STAGE_KEYS : DecCfg<128>::STAGE_KEYS,
+                                      di->num_sms);
     const size_t slots = static_cast<size_t>(BH) + DEC_MAX_CTAS - 1;
     float* part_o = static_cast<float*>(workspace);
     float2* part_ml = reinterpret_cast<float2*>(

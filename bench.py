@@ -37,6 +37,7 @@ DATASHEET_BF16_TFLOPS = 2250.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_NAME = "attn_fwd_sm100_kernel"
 SRC = os.path.join(ROOT, "exact_attention_127_b200", "csrc", "attn_fwd_sm100.cu")
+DECODE_SRC = os.path.join(ROOT, "exact_attention_127_b200", "csrc", "attn_decode.cuh")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
 L2_BYTES = 126 * 1024 * 1024
 
@@ -92,15 +93,28 @@ def source_digest() -> str:
     return hashlib.sha256(text[:cut] if cut >= 0 else text).hexdigest()
 
 
-def load_traffic(workload: str):
+def decode_source_digest() -> str:
+    """sha256 of the decode kernels' source file."""
+    with open(DECODE_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def load_traffic(workload: str, section: str | None = None):
     """DRAM bytes per launch from a committed ncu capture, or None when the
-    capture is missing, for another workload, or taken on older kernel source."""
+    capture is missing, for another workload, or taken on older kernel source.
+    section=None reads the forward kernel's record; "decode" reads the decode
+    stream kernel's, which carries the digest of its own source file."""
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f)
     except (OSError, ValueError):
         return None
-    if rec.get("kernel_source_sha256") != source_digest():
+    if section is not None:
+        rec = rec.get(section, {})
+        digest = decode_source_digest()
+    else:
+        digest = source_digest()
+    if rec.get("kernel_source_sha256") != digest:
         return None
     per = rec.get("per_launch_dram_bytes", {})
     val = per.get(workload)
@@ -660,7 +674,8 @@ def run_decode(args, w):
                        "l2": "K/V cache larger than L2" if flush is None else "L2 flushed"},
             "roofline": {"bound": "hbm", "achieved": value / world, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": value / world / peaks["hbm_gbs"],
-                         "traffic": load_traffic(w.name),
+                         "traffic": load_traffic(w.name, "decode"),
+                         "traffic_kernel": "decode_stream_kernel",
                          "peak_source": f"{peak_src} HBM copy (MEASURED_PEAKS.json)",
                          "kernel": "decode_stream_kernel + decode_combine_kernel (one call)",
                          "compulsory_bytes_per_launch": nbytes},

@@ -56,6 +56,20 @@ def test_traffic_ignored_when_kernel_changed(tmp_path, monkeypatch):
     assert bench.load_traffic("other") is None
 
 
+def test_decode_traffic_keyed_by_its_own_source(tmp_path, monkeypatch):
+    rec = {"kernel_source_sha256": bench.source_digest(), "per_launch_dram_bytes": {},
+           "decode": {"kernel_source_sha256": "0" * 64,
+                      "per_launch_dram_bytes": {"decode_b16h16_n8192_d128": 2.0}}}
+    p = tmp_path / "t.json"
+    p.write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(p))
+    assert bench.load_traffic("decode_b16h16_n8192_d128", "decode") is None
+    rec["decode"]["kernel_source_sha256"] = bench.decode_source_digest()
+    p.write_text(json.dumps(rec))
+    assert bench.load_traffic("decode_b16h16_n8192_d128", "decode") == 2.0
+    assert bench.load_traffic("decode_b16h16_n8192_d128") is None   # not in the forward record
+
+
 def test_oracle_sample_flops_counts_allowed_keys():
     w = inputs.WORKLOADS[inputs.HEADLINE]
     assert bench.oracle_sample_flops(w, [0, 9], 2) == 4 * 128 * (1 + 10) * 2

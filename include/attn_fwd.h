@@ -185,7 +185,8 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, float q_descale, f
 
 /*
  * attn_decode_workspace_bytes -- device workspace attn_decode needs for a shape
- * (the per-split partial results).  Returns 0 for invalid or empty shapes.
+ * ((B*H + 159) partial results of d fp32 values and an (m, l) pair: one per head
+ * and CTA that share keys).  Returns 0 for invalid or empty shapes.
  */
 size_t attn_decode_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
 
@@ -202,7 +203,10 @@ size_t attn_decode_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
  *   workspace: device scratch of at least attn_decode_workspace_bytes bytes,
  *         256-byte aligned, owned by the caller; its contents on entry are
  *         ignored.  Calls that overlap on the GPU must not share it.
- * Two kernels are enqueued on `stream` (split, then combine).  Same d, scale,
+ * Two kernels are enqueued on `stream`: a persistent stream kernel (one CTA per
+ * SM, each reading an equal share of the K/V cache once) that writes one partial
+ * per (head, CTA) to the workspace, then the combine.  A bounded wait that runs
+ * out sets ATTN_ERR_TIMEOUT in the device status word.  Same d, scale,
  * alignment and error conventions as attn_fwd; ATTN_ERR_WORKSPACE when the
  * workspace is missing, misaligned or too small; ATTN_ERR_OVERLAP when o, lse
  * or the workspace overlap an input or one another.
@@ -218,7 +222,7 @@ int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse
  * application owns every device allocation through its own pool, or a
  * latency-bound loop that must not allocate (cudaMalloc can synchronise the
  * device) once it runs.  It takes the same arguments as attn_decode minus the
- * workspace and allocates nothing: the per-split partial results go to a fixed
+ * workspace and allocates nothing: the partial results go to a fixed
  * static device buffer inside the library, attn_decode_noalloc_scratch_bytes()
  * = 8 MiB, which every GPU that loads the library holds until the process
  * exits.

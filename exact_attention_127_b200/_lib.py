@@ -75,6 +75,9 @@ def load_library():
     lib.attn_decode.restype = c_int
     lib.attn_fwd_test_wait_timeout.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
     lib.attn_fwd_test_wait_timeout.restype = c_int
+    lib.attn_decode_test_wait_timeout.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp,
+                                                  ctypes.c_size_t, vp]
+    lib.attn_decode_test_wait_timeout.restype = c_int
     lib.attn_status_str.argtypes = [c_int]
     lib.attn_status_str.restype = ctypes.c_char_p
     lib.attn_version.argtypes = []

@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
 decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const __nv_bfloat16* __restrict__ q, float* __restrict__ part_o,
                      float2* __restrict__ part_ml, int N, int sph, int per_cta, int total,
-                     float scale_log2, uint64_t wlim) {
+                     float scale_log2, uint64_t wlim, int withhold) {
     using C = DecCfg<D>;
     constexpr int CPL = D / 32;                  // output columns per lane
     constexpr int NCW = C::CONSUMERS;
@@ -103,7 +103,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(bp + C::FLAG_OFF);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int lo = blockIdx.x * per_cta;
-    const int hi = min(total, lo + per_cta);
+    const int hi = lo + min(per_cta, total - lo);        // lo < total for every CTA launched
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::NSTAGE; ++s) {
@@ -122,7 +122,8 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
             int it = 0;
-            for (int g = lo; g < hi; ++g, ++it) {
+            const int hi_load = withhold ? lo : hi;      // test hook: load nothing, so waits run out
+            for (int g = lo; g < hi_load; ++g, ++it) {
                 const int s = it % C::NSTAGE;
                 if (it >= C::NSTAGE &&
                     !mbar_wait(bar_empty(s), ((it / C::NSTAGE) - 1) & 1, abort_flag, wlim))
@@ -336,7 +337,8 @@ bool g_dec_smem_set[MAX_DEVICES][2];   // under g_mutex
 template <int D>
 int decode_launch(const CUtensorMap& mk, const CUtensorMap& mv, const __nv_bfloat16* q,
                   float* part_o, float2* part_ml, __nv_bfloat16* o, float* lse, int64_t BH,
-                  int N, const DecodePlan& pl, float scale_log2, int dev, cudaStream_t s) {
+                  int N, const DecodePlan& pl, float scale_log2, int dev, cudaStream_t s,
+                  uint64_t wait_limit_ns, int withhold) {
     auto kern = decode_stream_kernel<D>;
     constexpr int SMEM = DecCfg<D>::SMEM_BYTES;
     {
@@ -352,27 +354,17 @@ int decode_launch(const CUtensorMap& mk, const CUtensorMap& mv, const __nv_bfloa
         }
     }
     kern<<<pl.ctas, DecCfg<D>::THREADS, SMEM, s>>>(mk, mv, q, part_o, part_ml, N, pl.sph, pl.per_cta,
-                                            pl.total, scale_log2, WAIT_LIMIT_NS);
+                                            pl.total, scale_log2, wait_limit_ns, withhold);
     decode_combine_kernel<D><<<static_cast<unsigned>(BH), D, 0, s>>>(part_o, part_ml, o, lse, pl.sph,
                                                                     pl.per_cta);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
     return ATTN_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-size_t attn_decode_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {
-    bool empty = false;
-    if (decode_validate(B, H, N, d, 1.0f, &empty) != ATTN_OK) return 0;
-    if (empty) return 0;
-    return decode_ws_bytes(B * H, d);
-}
-
-int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+/* The decode call behind attn_decode and its timeout test hook. */
+int decode_impl(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
                 int64_t H, int64_t N, int64_t d, float scale, void* workspace,
-                size_t workspace_bytes, void* stream) {
+                size_t workspace_bytes, void* stream, uint64_t wait_limit_ns, int withhold) {
     bool empty = false;
     int st = decode_validate(B, H, N, d, scale, &empty);
     if (st != ATTN_OK || empty) return st;
@@ -415,9 +407,34 @@ int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse
     const auto* qb = static_cast<const __nv_bfloat16*>(q);
     auto* ob = static_cast<__nv_bfloat16*>(o);
     return d == 64 ? decode_launch<64>(mk, mv, qb, part_o, part_ml, ob, lse, BH, static_cast<int>(N), pl,
-                                       sl, dev, s)
+                                       sl, dev, s, wait_limit_ns, withhold)
                    : decode_launch<128>(mk, mv, qb, part_o, part_ml, ob, lse, BH, static_cast<int>(N), pl,
-                                        sl, dev, s);
+                                        sl, dev, s, wait_limit_ns, withhold);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t attn_decode_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {
+    bool empty = false;
+    if (decode_validate(B, H, N, d, 1.0f, &empty) != ATTN_OK) return 0;
+    if (empty) return 0;
+    return decode_ws_bytes(B * H, d);
+}
+
+int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+                int64_t H, int64_t N, int64_t d, float scale, void* workspace,
+                size_t workspace_bytes, void* stream) {
+    return decode_impl(q, k, v, o, lse, B, H, N, d, scale, workspace, workspace_bytes, stream,
+                       WAIT_LIMIT_NS, 0);
+}
+
+int attn_decode_test_wait_timeout(const void* q, const void* k, const void* v, void* o, float* lse,
+                                  int64_t B, int64_t H, int64_t N, int64_t d, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+    return decode_impl(q, k, v, o, lse, B, H, N, d, 0.125f, workspace, workspace_bytes, stream,
+                       TEST_WAIT_LIMIT_NS, 1);
 }
 
 }  // extern "C"

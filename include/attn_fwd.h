@@ -255,6 +255,17 @@ size_t attn_decode_noalloc_scratch_bytes(void);
 int attn_fwd_test_wait_timeout(const void* q, const void* k, const void* v, void* o, float* lse,
                                int64_t B, int64_t H, int64_t N, int64_t d, void* stream);
 
+/*
+ * attn_decode_test_wait_timeout -- the same test hook for the decode kernels.
+ * Takes attn_decode's arguments minus scale (and the same checks); the loader
+ * warp is told never to load K and V and every bounded wait is limited to
+ * 20 ms.  The waits run out, ATTN_ERR_TIMEOUT goes to the device status word
+ * and the kernels exit; o, lse and the workspace are left unspecified.
+ */
+int attn_decode_test_wait_timeout(const void* q, const void* k, const void* v, void* o, float* lse,
+                                  int64_t B, int64_t H, int64_t N, int64_t d, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
 /* attn_status_str -- a static, human-readable string for a status code. */
 const char* attn_status_str(int status);
 

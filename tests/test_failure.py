@@ -1,7 +1,8 @@
 """Failure detection without a GPU fault: every wait in the kernel is bounded.
 
-The test hook attn_fwd_test_wait_timeout runs the kernel with its K/V loads
-withheld and a 20 ms limit on each wait.  The waits run out, the kernel
+The test hooks attn_fwd_test_wait_timeout and attn_decode_test_wait_timeout run
+the forward and decode kernels with their K/V loads withheld and a 20 ms limit
+on each wait.  The waits run out, the kernel
 records ATTN_ERR_TIMEOUT in the device status word, frees its tensor memory
 and exits; the context stays usable for the next call.
 """
@@ -25,6 +26,10 @@ def test_hook_validates_arguments_on_host():
     fake = 0x10000
     rc = lib.attn_fwd_test_wait_timeout(fake, fake + 0x100000, fake + 0x200000, fake + 0x300000,
                                         fake + 0x400000, 1, 1, 128, 96, None)
+    assert rc == ATTN_ERR_HEADDIM
+    rc = lib.attn_decode_test_wait_timeout(fake, fake + 0x100000, fake + 0x200000, fake + 0x300000,
+                                           fake + 0x400000, 1, 1, 128, 96, fake + 0x500000, 1 << 20,
+                                           None)
     assert rc == ATTN_ERR_HEADDIM
 
 
@@ -55,3 +60,33 @@ def test_bounded_wait_runs_out_and_context_survives():
     O, L = oracle.attention_rows(qc, kc, vc, True, 1 / math.sqrt(64))
     assert np.abs(o2.cpu().reshape(2, 300, 64).double().numpy() - O).max() <= 2e-2
     assert np.abs(l2.cpu().reshape(2, 300).double().numpy() - L).max() <= 1e-3
+
+
+@pytest.mark.gpu
+def test_decode_bounded_wait_runs_out_and_context_survives():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    lib = attn.load_library()
+    assert attn.device_status(reset=True) == 0
+    B, H, N, d = 2, 3, 3000, 128
+    q, k, v = (t.cuda() for t in inputs.make_decode_qkv(B, H, N, d, 33))
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, dtype=torch.float32, device="cuda")
+    ws = torch.empty(attn.decode_workspace_bytes(B, H, N, d), dtype=torch.uint8, device="cuda")
+    t0 = time.perf_counter()
+    rc = lib.attn_decode_test_wait_timeout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                           lse.data_ptr(), B, H, N, d, ws.data_ptr(), ws.numel(),
+                                           torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    status = attn.device_status(reset=True)
+    elapsed = time.perf_counter() - t0
+    assert status == ATTN_ERR_TIMEOUT
+    assert elapsed < 10.0
+    assert attn.device_status(reset=True) == 0
+    # the next ordinary decode call runs normally and is correct
+    o2, l2 = attn.attn_decode(q, k, v)
+    torch.cuda.synchronize()
+    assert attn.device_status(reset=True) == 0
+    O, L = oracle.attention_qk(q.cpu(), k.cpu(), v.cpu(), 1.0 / math.sqrt(d))
+    assert np.abs(o2.cpu().reshape(B * H, 1, d).double().numpy() - O).max() <= 2e-2
+    assert np.abs(l2.cpu().reshape(B * H, 1).double().numpy() - L).max() <= 1e-3

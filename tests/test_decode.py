@@ -29,6 +29,12 @@ def test_decode_validation_on_host():
     assert lib.attn_decode_workspace_bytes(1, 2, 100, 80) == 0
     need = lib.attn_decode_workspace_bytes(16, 16, 8192, 128)
     assert need >= 16 * 16 * 128 * 4   # at least one fp32 partial per head
+    # one partial per (head, CTA) pair that shares keys: at most B*H + 159 of them
+    # (d fp32 values, 256-byte aligned, then an (m, l) pair each); independent of N
+    for B, H, N, d in [(16, 16, 8192, 128), (1, 1, 1, 64), (32, 32, 4096, 64)]:
+        slots = B * H + 159
+        expect = (slots * d * 4 + 255) // 256 * 256 + slots * 8
+        assert lib.attn_decode_workspace_bytes(B, H, N, d) == expect
 
 
 @pytest.fixture(scope="module")

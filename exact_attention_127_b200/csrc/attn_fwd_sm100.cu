@@ -1379,7 +1379,15 @@ int std_launch(const void* q, const void* k, const void* v, const StdParams& prm
         std_softmax_short_kernel<<<static_cast<unsigned>((rows + per - 1) / per),
                                    STD_SOFTMAX_THREADS, 0, stream>>>(prm);
     } else {
-        std_softmax_kernel<<<static_cast<unsigned>(rows), STD_SOFTMAX_THREADS, 0, stream>>>(prm);
+        const unsigned g = static_cast<unsigned>(rows);
+        if (prm.Np <= 4 * STD_SOFTMAX_THREADS * 4)
+            std_softmax_kernel<4><<<g, STD_SOFTMAX_THREADS, 0, stream>>>(prm);
+        else if (prm.Np <= 4 * STD_SOFTMAX_THREADS * 8)
+            std_softmax_kernel<8><<<g, STD_SOFTMAX_THREADS, 0, stream>>>(prm);
+        else if (prm.Np <= 4 * STD_SOFTMAX_THREADS * 16)
+            std_softmax_kernel<16><<<g, STD_SOFTMAX_THREADS, 0, stream>>>(prm);
+        else
+            std_softmax_kernel<STD_MAX_N / (4 * STD_SOFTMAX_THREADS)><<<g, STD_SOFTMAX_THREADS, 0, stream>>>(prm);
     }
     k3<<<dim3(tiles, prm.BH), STD_THREADS, smem3, stream>>>(mp, mv, prm);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;

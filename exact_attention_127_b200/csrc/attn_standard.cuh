@@ -128,10 +128,13 @@ std_qk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 }
 
 /* Kernel 2: one row per CTA -- row max, exponentials, row sum, P = e^{s-m}/l
- * written as bf16 over the row's first half, and LSE = m + ln l. */
+ * written as bf16 over the row's first half, and LSE = m + ln l.  VEC float4
+ * per thread covers rows of up to 1024 VEC scores; the smallest VEC that
+ * covers the row keeps registers, and so resident rows per SM, high.  Masked
+ * scores (causal, j > i) are not read: their P is written as 0. */
+template <int VEC>
 __global__ void __launch_bounds__(STD_SOFTMAX_THREADS)
 std_softmax_kernel(const StdParams p) {
-    constexpr int VEC = STD_MAX_N / (4 * STD_SOFTMAX_THREADS);   // float4 per thread, max
     __shared__ float red[STD_SOFTMAX_THREADS / 32];
     const int64_t row = blockIdx.x;
     const int bh = static_cast<int>(row / p.N), i = static_cast<int>(row % p.N);
@@ -144,7 +147,7 @@ std_softmax_kernel(const StdParams p) {
     for (int u = 0; u < VEC; ++u) {
         const int g = threadIdx.x + STD_SOFTMAX_THREADS * u;
         float4 t = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-        if (g < nvec) {
+        if (g < nvec && 4 * g < n_valid) {
             t = reinterpret_cast<const float4*>(srow)[g];
             const int e = 4 * g;
             if (e >= n_valid) t.x = -INFINITY;

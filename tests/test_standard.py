@@ -58,3 +58,28 @@ def test_standard_and_fused_agree_on_a_workload():
     assert attn.device_status(reset=True) == 0
     assert (o1.float() - o2.float()).abs().max().item() <= 2 * O_MAX_ABS
     assert (l1 - l2).abs().max().item() <= 2 * LSE_MAX_ABS
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("N,causal", [(2049, True), (4096, False), (4097, True), (8192, True),
+                                      (8193, False), (16384, True), (16385, True)])
+def test_standard_long_rows_sampled(N, causal):
+    """Rows longer than 2048 keys take the CTA-per-row softmax, instantiated for
+    4, 8, 16 or 32 float4 per thread by row length: each class and its edges,
+    checked on sampled rows (boundary rows plus seeded draws) of two heads."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    d = 64
+    q, k, v = inputs.make_qkv(1, 2, N, d, seed=400 + N)
+    o, lse = attn.attn_standard(q.cuda(), k.cuda(), v.cuda(), causal=causal)
+    torch.cuda.synchronize()
+    assert attn.device_status(reset=True) == 0
+    rng = np.random.default_rng(N)
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, N // 2, N - 2, N - 1],
+                                     rng.integers(0, N, 57)])).astype(np.int64)
+    O, L = oracle.attention_rows(q, k, v, causal, 1 / math.sqrt(d), rows=rows)
+    of = o.cpu().reshape(2, N, d)[:, torch.from_numpy(rows)].double().numpy()
+    lf = lse.cpu().reshape(2, N)[:, torch.from_numpy(rows)].double().numpy()
+    assert np.abs(of - O).max() <= O_MAX_ABS
+    assert np.linalg.norm(of - O) / np.linalg.norm(O) <= O_REL_L2
+    assert np.abs(lf - L).max() <= LSE_MAX_ABS

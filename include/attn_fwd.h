@@ -228,8 +228,8 @@ int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse
  * exits.
  *   - Shapes whose partials need more than that (attn_decode_workspace_bytes
  *     > 8 MiB; about (B*H + 159)*(d + 2)*4 bytes, i.e. any B*H beyond 15972
- *     at d = 128 or 31616 at d = 64) are rejected with ATTN_ERR_WORKSPACE before anything
- *     runs.
+ *     at d = 128 or 31616 at d = 64) are rejected with ATTN_ERR_WORKSPACE
+ *     before anything runs.
  *   - The buffer's device address is looked up on the first call on each
  *     device, with that device current; make that first call outside any
  *     stream capture.

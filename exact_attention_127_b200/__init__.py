@@ -10,10 +10,11 @@ keys (split-K/V).
 """
 from ._lib import (AttnError, attn_bwd, attn_decode, attn_fwd, attn_fwd_fp8, attn_fwd_host,
                    attn_standard, bwd_workspace_bytes, decode_workspace_bytes, device_status,
-                   fp8_workspace_bytes, header_functions, host_workspace_bytes, load_library,
-                   standard_workspace_bytes, status_str, version)
+                   fp8_workspace_bytes, fwd_schedule, header_functions, host_workspace_bytes,
+                   load_library, standard_workspace_bytes, status_str, version)
 
 __all__ = ["AttnError", "attn_bwd", "attn_decode", "attn_fwd", "attn_fwd_fp8", "attn_fwd_host",
            "attn_standard", "bwd_workspace_bytes", "fp8_workspace_bytes",
-           "decode_workspace_bytes", "device_status", "header_functions", "host_workspace_bytes",
-           "load_library", "standard_workspace_bytes", "status_str", "version"]
+           "decode_workspace_bytes", "device_status", "fwd_schedule", "header_functions",
+           "host_workspace_bytes", "load_library", "standard_workspace_bytes", "status_str",
+           "version"]

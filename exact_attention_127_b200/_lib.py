@@ -78,6 +78,9 @@ def load_library():
     lib.attn_decode_test_wait_timeout.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp,
                                                   ctypes.c_size_t, vp]
     lib.attn_decode_test_wait_timeout.restype = c_int
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    lib.attn_fwd_schedule.argtypes = [i64, i64, i64, c_int, c_int, i32p, i32p, i64]
+    lib.attn_fwd_schedule.restype = i64
     lib.attn_status_str.argtypes = [c_int]
     lib.attn_status_str.restype = ctypes.c_char_p
     lib.attn_version.argtypes = []
@@ -156,6 +159,26 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = F
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd")
     return out, lse
+
+
+def fwd_schedule(B: int, H: int, N: int, causal: bool, grid: int):
+    """The forward kernel's static schedule (host only, no GPU needed).
+
+    Returns (cta, slot): int32 tensors of B*H*ceil(N/256) entries; unit
+    u = bh*ceil(N/256) + pair runs on CTA cta[u] as its slot[u]-th unit.
+    """
+    n_units = B * H * ((N + 255) // 256)
+    cta = torch.full((max(n_units, 1),), -1, dtype=torch.int32)
+    slot = torch.full((max(n_units, 1),), -1, dtype=torch.int32)
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    rc = load_library().attn_fwd_schedule(B, H, N, int(bool(causal)), int(grid),
+                                          ctypes.cast(cta.data_ptr(), i32p),
+                                          ctypes.cast(slot.data_ptr(), i32p), cta.numel())
+    if rc < 0:
+        raise AttnError(int(rc), "attn_fwd_schedule")
+    if rc != n_units:
+        raise RuntimeError(f"attn_fwd_schedule visited {rc} units, expected {n_units}")
+    return cta[:n_units], slot[:n_units]
 
 
 def host_workspace_bytes(B: int, H: int, N: int, d: int) -> int:

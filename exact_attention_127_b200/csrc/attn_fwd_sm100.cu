@@ -32,8 +32,10 @@
  *   every K/V block and ping-pong on the tensor core (while one tile's softmax
  *   runs, the other tile's GEMMs run).  Causal: blocks above the diagonal are
  *   never loaded or computed; only the diagonal block is masked element-wise
- *   (the same page, section 6 table).  Units are ordered longest first and dealt to
- *   the persistent CTAs in snake order.
+ *   (the same page, section 6 table).  Causal units are grouped into mirror
+ *   pairs of equal total length, which keeps the persistent CTAs in step on a
+ *   few heads at a time (K/V read from HBM about once), and the last round's
+ *   worth is dealt longest first (see sched_unit).
  *
  * Every wait on an mbarrier is bounded (iterations and wall time); when one
  * runs out the CTA records ATTN_ERR_TIMEOUT in a device status word, raises an
@@ -116,6 +118,15 @@ struct FwdParams {
     uint64_t wait_limit_ns;  // bound on every mbarrier wait
     int withhold_kv;         // test hook: the producer never loads K/V, so waits run out
     float o_scale;           // e4m3 path: V's descale factor, applied to O at the end
+    /* causal schedule (plan_schedule): mirror-job rounds, then the tail */
+    int jobs_per_head;       // ceil(n_pairs / 2)
+    int mirror_rounds;       // rounds of one mirror job per CTA
+    int tail_bh0;            // first head with units in the tail
+    int tail_m0;             // jobs of head tail_bh0 below this index ran as mirror jobs
+    int tail_full;           // heads after tail_bh0 (all their units are in the tail)
+    int tail_a;              // tail units of the top tail_m0 pair indices
+    int tail_b;              // tail units of the middle pair indices (tail_bh0 included)
+    int tail_units;          // all tail units
 };
 
 __device__ int g_attn_status = 0;
@@ -562,38 +573,97 @@ struct Unit {
     int n[2];   // K/V blocks Q tile t needs (0 when the tile lies past N)
 };
 
-/* Causal units are ordered by decreasing work (pair index descending, heads
- * minor); non-causal units head-major so concurrent CTAs share K/V in L2. */
-template <bool CAUSAL>
-__device__ __forceinline__ Unit unit_at(int idx, const FwdParams& p) {
-    Unit u;
-    if (CAUSAL) {
-        u.pair = p.n_pairs - 1 - idx / p.BH;
-        u.bh = idx % p.BH;
-    } else {
-        u.bh = idx / p.n_pairs;
-        u.pair = idx % p.n_pairs;
-    }
+__host__ __device__ __forceinline__ void fill_unit(Unit& u, bool causal, const FwdParams& p) {
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         const int r0 = u.pair * UNIT_ROWS + t * BLOCK_M;
         if (r0 >= p.N) {
             u.n[t] = 0;
-        } else if (CAUSAL) {
+        } else if (causal) {
             const int last = r0 / BLOCK_N;          // the diagonal block of this tile
             u.n[t] = last + 1 < p.nkv ? last + 1 : p.nkv;
         } else {
             u.n[t] = p.nkv;
         }
     }
-    return u;
 }
 
-/* Snake deal: round r gives CTA c the unit r*G + c (r even) or r*G + G-1-c
- * (r odd), so each CTA's list mixes long and short units. */
-__device__ __forceinline__ int unit_index(int round) {
-    const int G = gridDim.x, c = blockIdx.x;
-    return round * G + ((round & 1) ? (G - 1 - c) : c);
+/* The s-th work unit of CTA `cta` out of `grid`.  Returns 1 with u filled, 0
+ * for an empty slot (skip it), -1 past the CTA's last unit.  Every warp role of
+ * a CTA walks the same sequence.
+ *
+ * Non-causal: every unit has the same work; units go round-robin in head-major
+ * order, so the CTAs of a round share the K/V of a few heads in L2.
+ *
+ * Causal (units need 2*pair + 1 and 2*pair + 2 K/V blocks for their two Q
+ * tiles, so they differ in length): a job is the mirror pair of units
+ * {P-1-m, m} of one head (P = n_pairs).  Its two units need
+ * 2(P-1-m) + 2 + 2m + 2 = 2P + 2 blocks in all, the same for every job, so in
+ * each of the first mirror_rounds rounds every CTA runs one job and all CTAs
+ * stay in step; the jobs of one round are those of a few consecutive heads, so
+ * each head's K/V blocks come from HBM once and then from L2.  The remaining
+ * units (at least one round's worth of jobs) are ordered longest first
+ * (pair index descending, head ascending) and dealt in snake order (round r
+ * gives CTA c the unit r*G + c when r is even, r*G + G-1-c when odd), which
+ * evens out the end of the launch.  plan_schedule sets the parameters. */
+__host__ __device__ __forceinline__ int sched_unit(int s, int cta, int grid, bool causal,
+                                                   const FwdParams& p, Unit& u) {
+    if (!causal) {
+        const int idx = s * grid + cta;
+        if (idx >= p.n_units) return -1;
+        u.bh = idx / p.n_pairs;
+        u.pair = idx - u.bh * p.n_pairs;
+        fill_unit(u, false, p);
+        return 1;
+    }
+    const int P = p.n_pairs;
+    if (s < 2 * p.mirror_rounds) {
+        const int job = (s >> 1) * grid + cta;
+        u.bh = job / p.jobs_per_head;
+        const int m = job - u.bh * p.jobs_per_head;
+        if (s & 1) {
+            if (2 * m == P - 1) return 0;       // the middle unit of an odd P stands alone
+            u.pair = m;
+        } else {
+            u.pair = P - 1 - m;
+        }
+    } else {
+        const int r = s - 2 * p.mirror_rounds;
+        const int i = r * grid + ((r & 1) ? (grid - 1 - cta) : cta);
+        if (i >= p.tail_units) return -1;
+        const int hf = p.tail_full, m0 = p.tail_m0, bh0 = p.tail_bh0;
+        if (i < p.tail_a) {                           // pairs P-1 .. P-m0: full heads only
+            u.pair = P - 1 - i / hf;
+            u.bh = bh0 + 1 + i % hf;
+        } else if (i < p.tail_a + p.tail_b) {         // pairs P-1-m0 .. m0: head bh0 too
+            const int k = i - p.tail_a;
+            u.pair = P - 1 - m0 - k / (hf + 1);
+            u.bh = bh0 + k % (hf + 1);
+        } else {                                      // pairs m0-1 .. 0: full heads only
+            const int k = i - p.tail_a - p.tail_b;
+            u.pair = m0 - 1 - k / hf;
+            u.bh = bh0 + 1 + k % hf;
+        }
+    }
+    fill_unit(u, true, p);
+    return 1;
+}
+
+/* Host side of the causal schedule: mirror rounds leave at least one round of
+ * jobs to the longest-first tail. */
+inline void plan_schedule(FwdParams& p, int grid) {
+    const int P = p.n_pairs;
+    p.jobs_per_head = (P + 1) / 2;
+    const int64_t njobs = static_cast<int64_t>(p.BH) * p.jobs_per_head;
+    const int64_t rounds = njobs / grid - 1;
+    p.mirror_rounds = rounds > 0 ? static_cast<int>(rounds) : 0;
+    const int64_t first = static_cast<int64_t>(p.mirror_rounds) * grid;   // first tail job
+    p.tail_bh0 = static_cast<int>(first / p.jobs_per_head);
+    p.tail_m0 = static_cast<int>(first % p.jobs_per_head);
+    p.tail_full = p.BH - 1 - p.tail_bh0;
+    p.tail_a = p.tail_m0 * p.tail_full;
+    p.tail_b = (P - 2 * p.tail_m0) * (p.tail_full + 1);
+    p.tail_units = 2 * p.tail_a + p.tail_b;
 }
 
 /* ------------------------------------------------------------------------ */
@@ -673,9 +743,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             int local = 0;            // units this CTA has started
             bool aborted = false;
             for (int r = 0;; ++r) {
-                const int idx = unit_index(r);
-                if (idx >= p.n_units) break;
-                const Unit u = unit_at<CAUSAL>(idx, p);
+                Unit u;
+                const int got = sched_unit(r, blockIdx.x, gridDim.x, CAUSAL, p, u);
+                if (got < 0) break;
+                if (got == 0) continue;
                 if (local > 0 && !mbar_wait_inl(bar_q_empty, (local - 1) & 1, abort_flag, wlim)) {
                     aborted = true;
                     break;
@@ -752,9 +823,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             int local = 0;
             bool aborted = false;
             for (int r = 0; !aborted; ++r) {
-                const int idx = unit_index(r);
-                if (idx >= p.n_units) break;
-                const Unit u = unit_at<CAUSAL>(idx, p);
+                Unit u;
+                const int got = sched_unit(r, blockIdx.x, gridDim.x, CAUSAL, p, u);
+                if (got < 0) break;
+                if (got == 0) continue;
                 const int n0 = u.n[0], n1 = u.n[1];
                 const int nmax = n0 > n1 ? n0 : n1;
                 if (!mbar_wait_inl(bar_q_full, local & 1, abort_flag, wlim)) { aborted = true; break; }
@@ -833,9 +905,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int tail = p.N & (BLOCK_N - 1);   // valid keys in the last block (0 = full)
 
         for (int r = 0;; ++r) {
-            const int idx = unit_index(r);
-            if (idx >= p.n_units) break;
-            const Unit u = unit_at<CAUSAL>(idx, p);
+            Unit u;
+            const int got = sched_unit(r, blockIdx.x, gridDim.x, CAUSAL, p, u);
+            if (got < 0) break;
+            if (got == 0) continue;
             const int n = t ? u.n[1] : u.n[0];   // (not u.n[t]: no local-memory copy of u)
             if (n == 0) continue;
             const int row = u.pair * UNIT_ROWS + t * BLOCK_M + row_in_tile;
@@ -1007,32 +1080,78 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 constexpr int MAX_DEVICES = 64;
 
+/* Per-device state.  What depends on the CUDA context (kernel attributes set
+ * with cudaFuncSetAttribute, the device address of a __device__ symbol) is
+ * keyed by the id of the context current on the calling thread: after a
+ * cudaDeviceReset, or with another context made current, it is set up again
+ * instead of being reused. */
 struct DeviceInfo {
     bool ready = false;
     int status = ATTN_OK;   // ATTN_ERR_DEVICE when the device is not CC 10.0
     int num_sms = 0;
-    bool smem_set[8] = {false, false, false, false, false, false, false, false};
+    unsigned long long ctx_id = 0;   // context the flags and addresses below belong to
+    bool ctx_known = false;
+    bool smem_set[8] = {};           // forward kernels: (FP8, D == 128, CAUSAL)
+    bool bwd_set[4] = {};            // backward kernels: (D == 128, CAUSAL)
+    bool dec_set[2] = {};            // decode stream kernels: D == 128
+    bool std_set[2] = {};            // standard-path GEMM kernels: D == 128
+    void* scratch = nullptr;         // device address of the no-alloc decode buffer
 };
 
 std::mutex g_mutex;
 DeviceInfo g_dev[MAX_DEVICES];
 EncodeTiledFn g_encode = nullptr;
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+
+/* A driver entry point by name (the library links the runtime only). */
+bool driver_entry(const char* name, void** fn) {
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint(name, fn, cudaEnableDefault, &qres) != cudaSuccess ||
+        qres != cudaDriverEntryPointSuccess || !*fn) {
+        cudaGetLastError();
+        return false;
+    }
+    return true;
+}
+
 int get_encode(EncodeTiledFn* fn) {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!g_encode) {
         void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult qres;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) !=
-                cudaSuccess ||
-            qres != cudaDriverEntryPointSuccess || !ptr) {
-            cudaGetLastError();
-            return ATTN_ERR_CUDA;
-        }
+        if (!driver_entry("cuTensorMapEncodeTiled", &ptr)) return ATTN_ERR_CUDA;
         g_encode = reinterpret_cast<EncodeTiledFn>(ptr);
     }
     *fn = g_encode;
     return ATTN_OK;
+}
+
+/* Process-unique id of the context current on this thread (caller holds
+ * g_mutex).  If none is current yet, a symbol lookup makes the runtime bind
+ * its primary context first. */
+int current_context_id(unsigned long long* id) {
+    if (!g_ctx_current || !g_ctx_get_id) {
+        void* a = nullptr;
+        void* b = nullptr;
+        if (!driver_entry("cuCtxGetCurrent", &a) || !driver_entry("cuCtxGetId", &b))
+            return ATTN_ERR_CUDA;
+        g_ctx_current = reinterpret_cast<CtxGetCurrentFn>(a);
+        g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(b);
+    }
+    CUcontext ctx = nullptr;
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS) return ATTN_ERR_CUDA;
+    if (!ctx) {
+        void* sym = nullptr;
+        if (cudaGetSymbolAddress(&sym, g_attn_status) != cudaSuccess) {
+            cudaGetLastError();
+            return ATTN_ERR_CUDA;
+        }
+        if (g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx) return ATTN_ERR_CUDA;
+    }
+    return g_ctx_get_id(ctx, id) == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 int device_info(int* dev_out, DeviceInfo** info_out) {
@@ -1053,9 +1172,21 @@ int device_info(int* dev_out, DeviceInfo** info_out) {
         di.num_sms = sms;
         di.ready = true;
     }
+    if (di.status != ATTN_OK) return di.status;
+    unsigned long long id = 0;
+    const int st = current_context_id(&id);
+    if (st != ATTN_OK) return st;
+    if (!di.ctx_known || di.ctx_id != id) {   // first call in this context: set up again
+        for (int i = 0; i < 8; ++i) di.smem_set[i] = false;
+        for (int i = 0; i < 4; ++i) di.bwd_set[i] = false;
+        for (int i = 0; i < 2; ++i) di.dec_set[i] = di.std_set[i] = false;
+        di.scratch = nullptr;
+        di.ctx_id = id;
+        di.ctx_known = true;
+    }
     *dev_out = dev;
     *info_out = &di;
-    return di.status;
+    return ATTN_OK;
 }
 
 /* 3-D view [B*H][N][d] of a bf16 tensor, box = 64 columns x 128 rows x 1 head,
@@ -1115,7 +1246,9 @@ int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
         }
     }
     const int grid = prm.n_units < di->num_sms ? prm.n_units : di->num_sms;
-    kern<<<grid, NUM_THREADS, SMEM, stream>>>(mq, mk, mv, prm);
+    FwdParams sp = prm;
+    plan_schedule(sp, grid);
+    kern<<<grid, NUM_THREADS, SMEM, stream>>>(mq, mk, mv, sp);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
     return ATTN_OK;
 }
@@ -1340,7 +1473,7 @@ int std_validate(int64_t B, int64_t H, int64_t N, int64_t d, float scale, bool* 
 
 template <int D>
 int std_launch(const void* q, const void* k, const void* v, const StdParams& prm,
-               EncodeTiledFn enc, cudaStream_t stream) {
+               EncodeTiledFn enc, DeviceInfo* di, cudaStream_t stream) {
     CUtensorMap mq, mk, mv, mp;
     int st;
     if ((st = encode_map(enc, &mq, q, prm.BH, prm.N, D)) != ATTN_OK) return st;
@@ -1366,10 +1499,19 @@ int std_launch(const void* q, const void* k, const void* v, const StdParams& prm
     const int smem3 = STD_PV_STAGES * stage + 16 * STD_PV_STAGES + 64 + 1024;
     auto k1 = std_qk_kernel<D>;
     auto k3 = std_pv_kernel<D>;
-    if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1) != cudaSuccess ||
-        cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, smem3) != cudaSuccess) {
-        cudaGetLastError();
-        return ATTN_ERR_LAUNCH;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        bool& set = di->std_set[D == 128 ? 1 : 0];
+        if (!set) {
+            if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1) !=
+                    cudaSuccess ||
+                cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, smem3) !=
+                    cudaSuccess) {
+                cudaGetLastError();
+                return ATTN_ERR_LAUNCH;
+            }
+            set = true;
+        }
     }
     const unsigned tiles = static_cast<unsigned>(prm.Np / BLOCK_M);
     k1<<<dim3(tiles, tiles, prm.BH), STD_THREADS, smem1, stream>>>(mq, mk, prm);
@@ -1432,7 +1574,7 @@ int std_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     prm.scale = scale;
     prm.wait_limit_ns = WAIT_LIMIT_NS;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return d == 64 ? std_launch<64>(q, k, v, prm, enc, s) : std_launch<128>(q, k, v, prm, enc, s);
+    return d == 64 ? std_launch<64>(q, k, v, prm, enc, di, s) : std_launch<128>(q, k, v, prm, enc, di, s);
 }
 
 #include "attn_bwd.cuh"
@@ -1449,15 +1591,23 @@ size_t bwd_ws_bytes(int64_t BH, int64_t N, int64_t d) {
 template <int D, bool CAUSAL>
 int bwd_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                const CUtensorMap& mdo, const __nv_bfloat16* o, const __nv_bfloat16* dout,
-               const float* lse, const BwdParams& prm, cudaStream_t stream) {
+               const float* lse, const BwdParams& prm, DeviceInfo* di, cudaStream_t stream) {
     auto kern = bwd_main_kernel<D, CAUSAL>;
     constexpr int SMEM = BwdCfg<D>::SMEM_BYTES;
-    // the register split adds up only with BWD_LAUNCH_REGS per thread (see attn_bwd.cuh)
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != BWD_LAUNCH_REGS ||
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess) {
-        cudaGetLastError();
-        return ATTN_ERR_LAUNCH;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        bool& set = di->bwd_set[(D == 128 ? 2 : 0) + (CAUSAL ? 1 : 0)];
+        if (!set) {
+            // the register split adds up only with BWD_LAUNCH_REGS per thread (see attn_bwd.cuh)
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != BWD_LAUNCH_REGS ||
+                cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
+                    cudaSuccess) {
+                cudaGetLastError();
+                return ATTN_ERR_LAUNCH;
+            }
+            set = true;
+        }
     }
     const int64_t prows = static_cast<int64_t>(prm.BH) * prm.Np;
     if (cudaMemsetAsync(prm.dq_acc, 0, static_cast<size_t>(prows) * D * 4, stream) != cudaSuccess)
@@ -1528,10 +1678,10 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     const auto* ob = static_cast<const __nv_bfloat16*>(o);
     const auto* db = static_cast<const __nv_bfloat16*>(dout);
     if (d == 64)
-        return causal ? bwd_launch<64, true>(mq, mk, mv, mdo, ob, db, lse, prm, s)
-                      : bwd_launch<64, false>(mq, mk, mv, mdo, ob, db, lse, prm, s);
-    return causal ? bwd_launch<128, true>(mq, mk, mv, mdo, ob, db, lse, prm, s)
-                  : bwd_launch<128, false>(mq, mk, mv, mdo, ob, db, lse, prm, s);
+        return causal ? bwd_launch<64, true>(mq, mk, mv, mdo, ob, db, lse, prm, di, s)
+                      : bwd_launch<64, false>(mq, mk, mv, mdo, ob, db, lse, prm, di, s);
+    return causal ? bwd_launch<128, true>(mq, mk, mv, mdo, ob, db, lse, prm, di, s)
+                  : bwd_launch<128, false>(mq, mk, mv, mdo, ob, db, lse, prm, di, s);
 }
 
 }  // namespace
@@ -1546,6 +1696,44 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
 int attn_fwd_test_wait_timeout(const void* q, const void* k, const void* v, void* o, float* lse,
                                int64_t B, int64_t H, int64_t N, int64_t d, void* stream) {
     return fwd_impl(q, k, v, o, lse, B, H, N, d, 0, 0.125f, stream, TEST_WAIT_LIMIT_NS, 1);
+}
+
+int64_t attn_fwd_schedule(int64_t B, int64_t H, int64_t N, int causal, int grid,
+                          int32_t* cta_of_unit, int32_t* slot_of_unit, int64_t capacity) {
+    bool empty = false;
+    const int st = validate_shape(B, H, N, 128, 1.0f, &empty);
+    if (st != ATTN_OK) return st;
+    if (empty) return 0;
+    if (grid < 1) return ATTN_ERR_SHAPE;
+    FwdParams prm;
+    memset(&prm, 0, sizeof(prm));
+    prm.N = static_cast<int>(N);
+    prm.BH = static_cast<int>(B * H);
+    prm.n_pairs = static_cast<int>((N + UNIT_ROWS - 1) / UNIT_ROWS);
+    prm.nkv = static_cast<int>((N + BLOCK_N - 1) / BLOCK_N);
+    prm.n_units = prm.BH * prm.n_pairs;
+    if (!cta_of_unit || !slot_of_unit) return ATTN_ERR_NULL;
+    if (capacity < prm.n_units) return ATTN_ERR_WORKSPACE;
+    if (grid > prm.n_units) grid = prm.n_units;
+    plan_schedule(prm, grid);
+    for (int64_t i = 0; i < prm.n_units; ++i) cta_of_unit[i] = slot_of_unit[i] = -1;
+    int64_t visits = 0;
+    for (int c = 0; c < grid; ++c) {
+        int slot = 0;
+        for (int s = 0;; ++s) {
+            Unit u;
+            const int got = sched_unit(s, c, grid, causal != 0, prm, u);
+            if (got < 0) break;
+            if (got == 0) continue;
+            ++visits;
+            if (u.bh < 0 || u.bh >= prm.BH || u.pair < 0 || u.pair >= prm.n_pairs)
+                return ATTN_ERR_SHAPE;   // a unit outside the problem: a scheduling bug
+            const int64_t idx = static_cast<int64_t>(u.bh) * prm.n_pairs + u.pair;
+            cta_of_unit[idx] = c;
+            slot_of_unit[idx] = slot++;
+        }
+    }
+    return visits;
 }
 
 size_t attn_fwd_fp8_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {

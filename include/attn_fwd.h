@@ -231,8 +231,11 @@ int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse
  *     at d = 128 or 31616 at d = 64) are rejected with ATTN_ERR_WORKSPACE
  *     before anything runs.
  *   - The buffer's device address is looked up on the first call on each
- *     device, with that device current; make that first call outside any
- *     stream capture.
+ *     device, with that device current, and again on the first call after
+ *     the current CUDA context changed (a cudaDeviceReset, or another context
+ *     made current): the address belongs to a context, so a cached one is
+ *     never reused in another.  Make such a first call outside any stream
+ *     capture.
  *   - Every call shares the one buffer, which keeps the last call's partials.
  *     Nothing in it has to start at zero (every partial is written before it
  *     is read), but calls that overlap on the GPU (other streams, other host
@@ -266,6 +269,25 @@ int attn_fwd_test_wait_timeout(const void* q, const void* k, const void* v, void
 int attn_decode_test_wait_timeout(const void* q, const void* k, const void* v, void* o, float* lse,
                                   int64_t B, int64_t H, int64_t N, int64_t d, void* workspace,
                                   size_t workspace_bytes, void* stream);
+
+/*
+ * attn_fwd_schedule -- host-only query of the forward kernel's static work
+ * schedule (no CUDA call; usable without a GPU).  The work is split into units
+ * of two 128-row Q tiles of one head: unit u = bh * ceil(N/256) + pair covers
+ * query rows [256*pair, 256*pair + 256) of head bh.  Persistent CTAs walk the
+ * units in a fixed order so that work is spread evenly ("GPU 学习日报 Day 21",
+ * section 6: parallelism over query row blocks; longest causal blocks first).
+ *   grid          : number of CTAs (attn_fwd uses min(SM count, units)).
+ *   cta_of_unit   : host, int32 [capacity], written: the CTA that runs unit u.
+ *   slot_of_unit  : host, int32 [capacity], written: u's position in that CTA's
+ *                   sequence (0 = first).
+ * Returns the number of units the CTAs visit (equal to B*H*ceil(N/256) when
+ * every unit runs once), or a negative attn_status_t: ATTN_ERR_SHAPE (shape,
+ * grid < 1, or a unit outside the problem), ATTN_ERR_NULL, ATTN_ERR_WORKSPACE
+ * (capacity below the unit count).  Head dimension does not change the order.
+ */
+int64_t attn_fwd_schedule(int64_t B, int64_t H, int64_t N, int causal, int grid,
+                          int32_t* cta_of_unit, int32_t* slot_of_unit, int64_t capacity);
 
 /* attn_status_str -- a static, human-readable string for a status code. */
 const char* attn_status_str(int status);

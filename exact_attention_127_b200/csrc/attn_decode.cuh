@@ -332,18 +332,16 @@ size_t decode_ws_bytes(int64_t BH, int64_t d) {
     return ((po + 255u) & ~static_cast<size_t>(255u)) + slots * sizeof(float2);
 }
 
-bool g_dec_smem_set[MAX_DEVICES][2];   // under g_mutex
-
 template <int D>
 int decode_launch(const CUtensorMap& mk, const CUtensorMap& mv, const __nv_bfloat16* q,
                   float* part_o, float2* part_ml, __nv_bfloat16* o, float* lse, int64_t BH,
-                  int N, const DecodePlan& pl, float scale_log2, int dev, cudaStream_t s,
+                  int N, const DecodePlan& pl, float scale_log2, DeviceInfo* di, cudaStream_t s,
                   uint64_t wait_limit_ns, int withhold) {
     auto kern = decode_stream_kernel<D>;
     constexpr int SMEM = DecCfg<D>::SMEM_BYTES;
     {
         std::lock_guard<std::mutex> lock(g_mutex);
-        bool& set = g_dec_smem_set[dev][D == 128 ? 1 : 0];
+        bool& set = di->dec_set[D == 128 ? 1 : 0];
         if (!set) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
                 cudaSuccess) {
@@ -407,9 +405,9 @@ int decode_impl(const void* q, const void* k, const void* v, void* o, float* lse
     const auto* qb = static_cast<const __nv_bfloat16*>(q);
     auto* ob = static_cast<__nv_bfloat16*>(o);
     return d == 64 ? decode_launch<64>(mk, mv, qb, part_o, part_ml, ob, lse, BH, static_cast<int>(N), pl,
-                                       sl, dev, s, wait_limit_ns, withhold)
+                                       sl, di, s, wait_limit_ns, withhold)
                    : decode_launch<128>(mk, mv, qb, part_o, part_ml, ob, lse, BH, static_cast<int>(N), pl,
-                                        sl, dev, s, wait_limit_ns, withhold);
+                                        sl, di, s, wait_limit_ns, withhold);
 }
 
 }  // namespace
@@ -452,26 +450,26 @@ constexpr size_t DECODE_STATIC_SCRATCH_BYTES = size_t(8) << 20;   // 8 MiB
 static __device__ __align__(256) unsigned char g_decode_scratch[DECODE_STATIC_SCRATCH_BYTES];
 
 namespace {
-std::mutex g_scratch_mutex;
-void* g_scratch_ptr[MAX_DEVICES] = {};
-
-/* Device address of g_decode_scratch on the current device.  In host code the
- * array's name only stands in for the symbol, so the address is looked up once
- * per device (with that device current) and cached. */
+/* Device address of g_decode_scratch in the context current on this thread.
+ * In host code the array's name only stands in for the symbol (it is not a
+ * device address), so the address is looked up with cudaGetSymbolAddress once
+ * per device and context, with that device current, and cached; a context
+ * reset or another current context leads to a fresh lookup (device_info). */
 int scratch_address(void** out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return ATTN_ERR_CUDA; }
-    if (dev < 0 || dev >= MAX_DEVICES) return ATTN_ERR_DEVICE;
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_ptr[dev]) {
+    DeviceInfo* di = nullptr;
+    const int st = device_info(&dev, &di);
+    if (st != ATTN_OK) return st;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!di->scratch) {
         void* ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || !ptr) {
             cudaGetLastError();
             return ATTN_ERR_CUDA;
         }
-        g_scratch_ptr[dev] = ptr;
+        di->scratch = ptr;
     }
-    *out = g_scratch_ptr[dev];
+    *out = di->scratch;
     return ATTN_OK;
 }
 }  // namespace

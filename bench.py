@@ -9,9 +9,13 @@ TFLOP/s with FLOPs = 4*B*H*N^2*d / 2 (causal), inputs resident in HBM.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...      # the fp64 CPU oracle, timed
 
-With N > 1 (launched by torch.distributed.run) every rank runs its own batch
-(seed + rank): the work shards by independent problems, there is no data-path
-collective, and scaling is weak.  Rank 0 prints one JSON line.
+With N > 1 (``--gpus N`` starts N ranks through torch.distributed.run unless
+it already runs under it) the heads are split over the ranks: by default each
+rank runs one batch block of an N-times larger problem (block r seeded with
+seed + 1000*r; weak scaling), with ``--scaling strong`` the workload's own heads
+are split into contiguous ranges.  Heads are independent, so there is no
+data-path collective; ``--gather`` also times an NCCL all-gather of O and LSE.
+Rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
@@ -271,15 +275,39 @@ def run_reference(args, w):
     return 0
 
 
-def config_of(w, world):
+def config_of(w, world, scaling="weak"):
+    BH = w.B * w.H
+    if world > 1 and scaling == "weak":
+        per_rank = (f"global problem [{world * w.B}, {w.H}, {w.N}, {w.d}]: rank r runs heads "
+                    f"[r*{BH}, (r+1)*{BH}) (batch block r, seed + 1000*r)")
+    elif world > 1:
+        per_rank = (f"global problem [{w.B}, {w.H}, {w.N}, {w.d}] (seed {w.seed}): rank r runs a "
+                    f"contiguous range of about {BH / world:.1f} of its {BH} heads")
+    else:
+        per_rank = "all heads on one GPU"
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
             "scale": w.scale, "seed": w.seed, "inputs": "bf16; " + (
                 "Q,K ~ N(0,16), V ~ U(-1,1)" if w.v_dist == "uniform" else "Q,K,V ~ N(0,1)"),
-            "per_rank": "one independent batch per rank (seed + 1000*rank)",
-            "parallelism": f"dp{world}" if world > 1 else "single GPU",
+            "per_rank": per_rank,
+            "parallelism": f"heads split over {world} GPUs" if world > 1 else "single GPU",
             "l2": ("inputs larger than L2 (q,k,v %.0f MB per step)" % (
                 3 * 2 * w.B * w.H * w.N * w.d / 1e6))
             if 3 * 2 * w.B * w.H * w.N * w.d > L2_BYTES else "L2 flushed between steps"}
+
+
+def rank_inputs(w, world, rank, scaling):
+    """This rank's q, k, v head slices ([count, N, d] CPU bf16) and the global
+    head count.  weak: the global problem is `world` batch blocks of the
+    workload, block r seeded with seed + 1000*r, and rank r owns block r.
+    strong: the global problem is the workload itself, split by head_range."""
+    from exact_attention_127_b200 import shard
+    if scaling == "weak" or world == 1:
+        q, k, v = _inputs.make_qkv(w.B, w.H, w.N, w.d, rank_seed(w.seed, rank), w.qk_std,
+                                   w.v_dist)
+        flat = [t.reshape(w.B * w.H, w.N, w.d) for t in (q, k, v)]
+        return flat, w.B * w.H * world
+    q, k, v = _inputs.workload_inputs(w)
+    return [shard.head_slice(t, world, rank).clone() for t in (q, k, v)], w.B * w.H
 
 
 def run_cuda(args, w):
@@ -287,8 +315,12 @@ def run_cuda(args, w):
     import torch.distributed as dist
 
     import exact_attention_127_b200 as attn
+    from exact_attention_127_b200 import shard
 
     rank, local, world = dist_env()
+    if world > 1 and torch.cuda.device_count() < world:
+        raise SystemExit(f"{world} ranks need {world} visible GPUs; "
+                         f"found {torch.cuda.device_count()}")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -296,24 +328,27 @@ def run_cuda(args, w):
                                 device_id=dev)
     attn.load_library()
 
-    q, k, v = _inputs.make_qkv(w.B, w.H, w.N, w.d, rank_seed(w.seed, rank), w.qk_std, w.v_dist)
+    (q, k, v), n_heads = rank_inputs(w, world, rank, args.scaling)
+    count = q.shape[0]
     qd, kd, vd = (t.to(dev) for t in (q, k, v))
     o = torch.empty_like(qd)
-    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    lse = torch.empty((count, w.N), dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(dev)
     flush = None
     big_enough = 3 * qd.numel() * 2 > L2_BYTES
     if not big_enough:
         flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
-    def step():
-        if flush is not None:
-            flush.fill_(1.0)   # evict L2 between timed iterations
-        attn.attn_fwd(qd, kd, vd, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
+    def fwd():
+        if count:
+            shard.attn_fwd_heads(qd, kd, vd, causal=w.causal, scale=w.scale, out=o, lse=lse,
+                                 stream=stream)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            step()
+            if flush is not None:
+                flush.fill_(1.0)   # evict L2 between iterations
+            fwd()
     stream.synchronize()
     if attn.device_status(reset=True, stream=stream) != 0:
         raise RuntimeError("kernel reported a device-side error during warm-up")
@@ -328,63 +363,111 @@ def run_cuda(args, w):
     with torch.cuda.stream(stream):
         for i in range(args.steps):
             if flush is not None:
-                flush.fill_(1.0)
+                flush.fill_(1.0)   # outside the events: a step is the forward call alone
             starts[i].record(stream)
-            attn.attn_fwd(qd, kd, vd, causal=w.causal, scale=w.scale, out=o, lse=lse,
-                          stream=stream)
+            fwd()
             ends[i].record(stream)
     stream.synchronize()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     sampler.stop()
-    launches = args.steps
+    launches = args.steps if count else 0
     kernel_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = starts[0].elapsed_time(ends[-1])
-    ms_step = total_ms / args.steps
     ms_kernel = sum(kernel_ms) / len(kernel_ms)
+    if flush is None:
+        ms_step = starts[0].elapsed_time(ends[-1]) / args.steps   # back-to-back steps
+    else:
+        ms_step = ms_kernel          # L2 flushed between steps: the steps' own time
     status = attn.device_status(reset=True, stream=stream)
     if status != 0:
         raise RuntimeError(f"kernel reported device status {status}")
 
-    # ---- end to end: host (pinned) buffers through the C ABI host entry point
-    qp, kp, vp = (t.pin_memory() for t in (q, k, v))
-    op = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
-    lp = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
-    ws = torch.empty(attn.host_workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
-    e2e_steps = max(1, min(args.steps, args.e2e_steps))
-    for _ in range(min(2, args.warmup)):
-        attn.attn_fwd_host(qp, kp, vp, w.causal, w.scale, out=op, lse=lp, workspace=ws,
-                           device=dev, stream=stream, synchronize=True)
-    if world > 1:
+    # ---- latency of one call (host call + launch + kernel), for launch-bound shapes
+    lat_us = None
+    if w.flops() < 1e9 and count:
+        host = []
+        for _ in range(args.latency_calls):
+            t0 = time.perf_counter()
+            fwd()
+            stream.synchronize()
+            host.append((time.perf_counter() - t0) * 1e6)
+        lat_us = {"call_median_us": statistics.median(host),
+                  "kernel_median_us": 1e3 * statistics.median(kernel_ms),
+                  "calls": args.latency_calls,
+                  "what": "host wall time of attn_fwd + stream synchronize, one call at a time"}
+
+    # ---- optional gather of every rank's O and LSE onto all ranks (NCCL all-gather)
+    gather = None
+    if args.gather and world > 1:
+        for _ in range(2):
+            shard.gather_heads(o, lse, n_heads)
+        torch.cuda.synchronize(dev)
         dist.barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        attn.attn_fwd_host(qp, kp, vp, w.causal, w.scale, out=op, lse=lp, workspace=ws,
-                           device=dev, stream=stream, synchronize=False)
-    e1.record(stream)
-    stream.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if attn.device_status(reset=True, stream=stream) != 0:
-        raise RuntimeError("kernel reported a device-side error in the e2e leg")
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for _ in range(args.steps):
+            o_all, lse_all = shard.gather_heads(o, lse, n_heads)
+        g1.record()
+        torch.cuda.synchronize(dev)
+        (g_ms,) = reduce_max([g0.elapsed_time(g1) / args.steps], dev)
+        nbytes = n_heads * w.N * (w.d * 2 + 4)
+        gather = {"ms_per_step": g_ms, "bytes_gathered": nbytes,
+                  "what": "NCCL all-gather of every rank's O and LSE slices, timed after the "
+                          "forward steps; not part of value"}
+
+    # ---- end to end: host (pinned) buffers through the C ABI host entry point
+    e2e_ms, h2d, d2h = None, 0, 0
+    if count:
+        qp, kp, vp = (t.reshape(1, count, w.N, w.d).pin_memory() for t in (q, k, v))
+        op = torch.empty(qp.shape, dtype=torch.bfloat16).pin_memory()
+        lp = torch.empty((1, count, w.N), dtype=torch.float32).pin_memory()
+        ws = torch.empty(attn.host_workspace_bytes(1, count, w.N, w.d), dtype=torch.uint8,
+                         device=dev)
+        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+        for _ in range(min(2, args.warmup)):
+            attn.attn_fwd_host(qp, kp, vp, w.causal, w.scale, out=op, lse=lp, workspace=ws,
+                               device=dev, stream=stream, synchronize=True)
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            attn.attn_fwd_host(qp, kp, vp, w.causal, w.scale, out=op, lse=lp, workspace=ws,
+                               device=dev, stream=stream, synchronize=False)
+        e1.record(stream)
+        stream.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / e2e_steps
+        h2d = 3 * qp.numel() * 2
+        d2h = op.numel() * 2 + lp.numel() * 4
+        if attn.device_status(reset=True, stream=stream) != 0:
+            raise RuntimeError("kernel reported a device-side error in the e2e leg")
+    elif world > 1:
+        dist.barrier()
+    if e2e_ms is None:
+        e2e_ms = 0.0
 
     ms_max, kern_max, e2e_max = reduce_max([ms_step, ms_kernel, e2e_ms], dev)
 
-    flops = w.flops()
-    value = aggregate_value(flops, world, ms_max)
+    # useful FLOPs of every rank's heads (a head of the workload: flops / (B*H))
+    flops_per_head = w.flops() / (w.B * w.H)
+    total_flops = flops_per_head * n_heads
+    value = total_flops / (ms_max * 1e-3) / 1e12
     line = None
     if rank == 0:
         peaks, peak_src = load_peaks()
-        achieved = flops / (kern_max * 1e-3) / 1e12
-        traffic = load_traffic(w.name)
+        rank_flops = flops_per_head * count
+        achieved = rank_flops / (kern_max * 1e-3) / 1e12
+        traffic = load_traffic(w.name) if world == 1 else None
         clocks = sampler.summary()
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": config_of(w, world),
+            "higher_is_better": True, "scaling": args.scaling if world > 1 else "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": config_of(w, world, args.scaling),
             "roofline": {
                 "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
@@ -394,23 +477,34 @@ def run_cuda(args, w):
                 "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
                 "frac_of_datasheet_2250": achieved / DATASHEET_BF16_TFLOPS,
                 "kernel": KERNEL_NAME, "kernel_ms": kern_max,
-                "algorithmic_flops_per_launch": flops,
-                "compulsory_bytes_per_launch": w.compulsory_bytes(),
+                "algorithmic_flops_per_launch": rank_flops,
+                "compulsory_bytes_per_launch": w.compulsory_bytes() * count // (w.B * w.H),
             },
-            "e2e": {"value": aggregate_value(flops, world, e2e_max), "unit": UNIT,
-                    "ms_per_step": e2e_max,
-                    "h2d_bytes_per_step": 3 * q.numel() * 2,
-                    "d2h_bytes_per_step": q.numel() * 2 + w.B * w.H * w.N * 4,
+            "e2e": {"value": total_flops / (e2e_max * 1e-3) / 1e12 if e2e_max else None,
+                    "unit": UNIT, "ms_per_step": e2e_max,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "path": "attn_fwd_host (pinned host buffers, copies + kernel on one stream)"},
             "gpu_launches": launches,
             "clocks": clocks,
         }
+        if flush is not None:
+            line["hbm"] = {"achieved_gbs": w.compulsory_bytes() / (kern_max * 1e-3) / 1e9,
+                           "peak_gbs": peaks["hbm_gbs"],
+                           "frac": w.compulsory_bytes() / (kern_max * 1e-3) / 1e9
+                           / peaks["hbm_gbs"],
+                           "what": "compulsory bytes (q, k, v read, o, lse written once) per "
+                                   "launch over the launch time, L2 flushed before each launch"}
+        if lat_us is not None:
+            line["latency"] = lat_us
+        if gather is not None:
+            line["gather"] = gather
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            cpu = time_oracle(w, q, k, v, target_s=args.cpu_seconds)
+            qf, kf, vf = (t.reshape(w.B, w.H, w.N, w.d) for t in (q, k, v))
+            cpu = time_oracle(w, qf, kf, vf, target_s=args.cpu_seconds)
             cpu.pop("rows")
             cpu.pop("heads")
             line["cpu_baseline"] = cpu
@@ -701,6 +795,33 @@ def run_decode(args, w):
     return 0
 
 
+def free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def relaunch(argv, n: int, limit_s: float = 3600.0) -> int:
+    """`--gpus N` without a launcher: start N ranks of this script through
+    torch.distributed.run on 127.0.0.1 and return their exit status.  The
+    ranks' own process-group timeout ends a stuck collective; limit_s bounds
+    the whole run as a last resort (the process group is killed)."""
+    import signal
+    import subprocess
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1",
+           "--master-port", str(free_port()), os.path.abspath(__file__), *argv]
+    proc = subprocess.Popen(cmd, start_new_session=True)
+    try:
+        return proc.wait(timeout=limit_s)
+    except subprocess.TimeoutExpired:
+        os.killpg(proc.pid, signal.SIGKILL)
+        proc.wait()
+        sys.stderr.write(f"bench: {n} ranks did not finish within {limit_s:.0f} s\n")
+        return 1
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -722,6 +843,13 @@ def main(argv=None):
                     help="fused kernel (default) or the unfused three-kernel path for comparison")
     ap.add_argument("--batch", type=int, default=None,
                     help="override B of the workload (smaller cases for profiler captures)")
+    ap.add_argument("--scaling", default="weak", choices=["weak", "strong"],
+                    help="N > 1: weak = each rank runs one batch block of an N-times larger "
+                         "problem (default); strong = the workload's heads split over the ranks")
+    ap.add_argument("--gather", action="store_true",
+                    help="N > 1: also time an NCCL all-gather of every rank's O and LSE")
+    ap.add_argument("--latency-calls", type=int, default=200,
+                    help="calls timed one at a time for the latency line of small workloads")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -738,6 +866,8 @@ def main(argv=None):
         import dataclasses
         w = dataclasses.replace(w, B=args.batch, name=f"{w.name}@B{args.batch}")
     _, _, world = dist_env()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return relaunch(argv if argv is not None else sys.argv[1:], args.gpus)
     if world != args.gpus:
         sys.stderr.write(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE\n")
     if args.impl == "reference":

@@ -127,3 +127,104 @@ def test_reference_arm_under_two_ranks_prints_one_line():
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["value"] > 0
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["cpu_baseline"]["kind"] == "oracle"
+
+
+# ---------------------------------------------------------------------------
+# One problem split over ranks by heads (exact_attention_127_b200.shard)
+# ---------------------------------------------------------------------------
+from exact_attention_127_b200 import shard  # noqa: E402
+
+
+@pytest.mark.parametrize("n_heads", [0, 1, 5, 16, 64, 1024, 1031])
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
+def test_head_range_partitions(n_heads, world):
+    ranges = [shard.head_range(n_heads, world, r) for r in range(world)]
+    assert ranges[0][0] == 0 and ranges[-1][1] == n_heads
+    for (a, b), (c, _) in zip(ranges, ranges[1:]):
+        assert b == c                                    # contiguous, in rank order
+    sizes = [b - a for a, b in ranges]
+    assert max(sizes) - min(sizes) <= 1 and sorted(sizes, reverse=True) == sizes
+
+
+def test_head_range_rejects_bad_arguments():
+    for args in ((4, 0, 0), (4, 2, 2), (4, 2, -1), (-1, 2, 0)):
+        with pytest.raises(ValueError):
+            shard.head_range(*args)
+
+
+def test_strong_split_slices_concatenate_to_the_problem():
+    w = inputs.WORKLOADS["tiny_n128_d64"]
+    w = type(w)(**{**w.__dict__, "B": 2, "H": 3})
+    full = [t.reshape(6, w.N, w.d) for t in inputs.workload_inputs(w)]
+    for world in (1, 2, 4):
+        parts = [bench.rank_inputs(w, world, r, "strong") for r in range(world)]
+        assert all(n == 6 for _, n in parts)
+        for i in range(3):
+            cat = torch.cat([p[0][i] for p in parts])
+            assert torch.equal(cat.view(torch.int16), full[i].view(torch.int16))
+
+
+def test_weak_split_gives_each_rank_its_own_block():
+    w = inputs.WORKLOADS["tiny_n128_d64"]
+    (q0, _, _), n0 = bench.rank_inputs(w, 2, 0, "weak")
+    (q1, _, _), n1 = bench.rank_inputs(w, 2, 1, "weak")
+    assert n0 == n1 == 2 * w.B * w.H
+    ref = inputs.make_qkv(w.B, w.H, w.N, w.d, bench.rank_seed(w.seed, 1))[0]
+    assert torch.equal(q1.view(torch.int16), ref.reshape(q1.shape).view(torch.int16))
+    assert not torch.equal(q0, q1)
+
+
+def _gather_worker(rank, world, port, out):
+    """Each rank computes its heads' O and LSE with the fp64 oracle (the CPU
+    stand-in for the kernel), rounds them like the kernel's outputs, and
+    gathers; every rank must end with the one-rank layout."""
+    import oracle
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        B, H, N, d = 1, 5, 40, 8
+        q, k, v = inputs.make_qkv(B, H, N, d, seed=9)
+        qs, ks, vs = (shard.head_slice(t, world, rank) for t in (q, k, v))
+        c = qs.shape[0]
+        if c:
+            O, L = oracle.attention(qs.view(1, c, N, d), ks.view(1, c, N, d),
+                                    vs.view(1, c, N, d), True, 0.3)
+            o_loc = torch.from_numpy(O).reshape(c, N, d).to(torch.bfloat16)
+            l_loc = torch.from_numpy(L).reshape(c, N).to(torch.float32)
+        else:
+            o_loc = torch.empty((0, N, d), dtype=torch.bfloat16)
+            l_loc = torch.empty((0, N), dtype=torch.float32)
+        o_all, l_all = shard.gather_heads(o_loc, l_loc, B * H)
+        O1, L1 = oracle.attention(q, k, v, True, 0.3)
+        o_ref = torch.from_numpy(O1).reshape(B * H, N, d).to(torch.bfloat16)
+        l_ref = torch.from_numpy(L1).reshape(B * H, N).to(torch.float32)
+        out[rank] = (torch.equal(o_all.view(torch.int16), o_ref.view(torch.int16)) and
+                     torch.equal(l_all.view(torch.int32), l_ref.view(torch.int32)) and
+                     o_all.dtype == torch.bfloat16)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_gather_heads_matches_one_rank_layout(world):
+    """Heads split 3/2 (world 2) or 2/2/1 (world 3): the gathered O and LSE equal
+    the one-rank result byte for byte on every rank."""
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_gather_worker, args=(world, port, out), nprocs=world, join=True)
+        assert [out[r] for r in range(world)] == [True] * world
+
+
+def test_bench_gpus_2_starts_its_own_ranks():
+    """`bench.py --gpus 2` run plainly (no launcher) starts two ranks itself."""
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+           "--workload", "tiny_n128_d64", "--steps", "2", "--warmup", "3",
+           "--ref-step-seconds", "0.05"]
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    res = subprocess.run(cmd, capture_output=True, text=True, timeout=240, cwd=ROOT, env=env)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    assert json.loads(lines[0])["n_gpus"] == 2

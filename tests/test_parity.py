@@ -151,9 +151,9 @@ def test_large_logits(attn, causal):
 
 @pytest.mark.parametrize("N", [1024, 1100])
 def test_large_logits_d64(attn, N):
-    """d = 64, non-causal, peaked softmax.  An even number of 128-row Q tiles
-    (N = 1024, and 1100 with a ragged tail) runs the three-S-buffer pipeline,
-    including its rescale path."""
+    """d = 64, non-causal, peaked softmax: the rescale path of the d = 64 kernel
+    on an even number of 128-row Q tiles (N = 1024) and with a ragged tail
+    (N = 1100)."""
     q, k, v = inputs.make_qkv(1, 3, N, 64, seed=14, qk_std=4.0, v_dist="uniform")
     _full_check(attn, q, k, v, False, label=f"large logits d64 N={N}")
 

@@ -415,13 +415,14 @@ __device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
 /* 2^x for a pair of values on the FMA/ALU pipes, to relieve the MUFU unit.
  * Range reduction (Cody-Waite style): x = n + f with n = round(x), obtained by
  * adding and subtracting 1.5 * 2^23 in fp32, and f in [-1/2, 1/2].  2^f is the
- * degree-3 polynomial with minimax relative error on [-1/2, 1/2] (Remez
- * exchange; coefficients and the fit in fit_exp2_poly.py next to this file;
- * max relative error 7.5e-5, far below the bf16 rounding of P).  2^n is
- * applied by adding n to the exponent field: the low mantissa bits of
- * x + 1.5 * 2^23 hold n, so shifting its bit pattern left by 23 yields n << 23.
- * x is clamped at -125 so the exponent stays normal (2^-125 is negligible next
- * to a row whose largest term is >= 1). */
+ * degree-3 polynomial with minimax relative error on [-1/2, 1/2], from a Remez
+ * exchange in fp64 with the coefficients rounded to fp32: max relative error
+ * 7.5e-5 over the fp32 evaluation, far below the bf16 rounding of P (a CPU test
+ * re-evaluates this arithmetic and checks the bound).  2^n is applied by
+ * adding n to the exponent field: the low mantissa bits of x + 1.5 * 2^23 hold
+ * n, so shifting its bit pattern left by 23 yields n << 23.  x is clamped at
+ * -125 so the exponent stays normal (2^-125 is negligible next to a row whose
+ * largest term is >= 1). */
 constexpr float EXP2_ROUND = 12582912.0f;          // 1.5 * 2^23
 constexpr float EXP2_C0 = 9.999280572e-01f;
 constexpr float EXP2_C1 = 6.932609677e-01f;

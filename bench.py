@@ -487,13 +487,14 @@ def run_cuda(args, w):
             "gpu_launches": launches,
             "clocks": clocks,
         }
-        if flush is not None:
-            line["hbm"] = {"achieved_gbs": w.compulsory_bytes() / (kern_max * 1e-3) / 1e9,
-                           "peak_gbs": peaks["hbm_gbs"],
-                           "frac": w.compulsory_bytes() / (kern_max * 1e-3) / 1e9
-                           / peaks["hbm_gbs"],
-                           "what": "compulsory bytes (q, k, v read, o, lse written once) per "
-                                   "launch over the launch time, L2 flushed before each launch"}
+        rank_bytes = w.compulsory_bytes() * count // (w.B * w.H)
+        gbs = rank_bytes / (kern_max * 1e-3) / 1e9
+        line["hbm"] = {"achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
+                       "frac": gbs / peaks["hbm_gbs"],
+                       "what": "compulsory bytes (q, k, v read, o, lse written once) per launch "
+                               "over the launch time"
+                               + ("; L2 flushed before each launch" if flush is not None else
+                                  "; inputs larger than L2")}
         if lat_us is not None:
             line["latency"] = lat_us
         if gather is not None:

@@ -267,25 +267,30 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
 /* The MMA statements carry no memory clobber: they touch no memory the compiler
  * tracks, and as volatile asm they stay ordered with the (clobbering) waits,
  * fences and commits around them. */
+/* `leader` selects the one thread that issues: the MMA warp runs its loop with
+ * all 32 lanes (so the descriptor arithmetic is warp-uniform) and lane 0
+ * issues every MMA and every commit (a commit tracks the MMAs of the thread
+ * that issues it). */
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
+                                       uint32_t idesc, uint32_t accumulate, uint32_t leader = 1u) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+        "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 e, %5, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(leader));
 }
 
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
+                                       uint32_t idesc, uint32_t accumulate, uint32_t leader = 1u) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
+        "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 e, %5, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(leader));
 }
 
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                 ::"r"(bar)
+__device__ __forceinline__ void mma_commit(uint32_t bar, uint32_t leader = 1u) {
+    asm volatile("{\n\t.reg .pred e;\n\tsetp.ne.b32 e, %1, 0;\n\t"
+                 "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
+                 ::"r"(bar), "r"(leader)
                  : "memory");
 }
 
@@ -293,11 +298,12 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
  * the first 16 columns of Q and K; k-step kk starts (kk/4) swizzle atoms plus
  * (kk%4)*32 bytes further, which only moves the start-address field. */
 template <int D>
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc) {
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc,
+                                         uint32_t leader = 1u) {
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
         const uint64_t off = static_cast<uint64_t>(((kk >> 2) * CHUNK_BYTES + (kk & 3) * 32) >> 4);
-        mma_ss(d_tmem, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
+        mma_ss(d_tmem, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u, leader);
     }
 }
 
@@ -305,12 +311,13 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t a0, uint64_t 
  * P is bf16 in TMEM (keys 2c, 2c+1 in column c); b0 describes V's first 16
  * keys (MN-major: 16 keys = 2048 bytes further per k-step). */
 __device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, uint64_t b0,
-                                              uint32_t idesc, uint32_t acc_first, int half) {
+                                              uint32_t idesc, uint32_t acc_first, int half,
+                                              uint32_t leader) {
 #pragma unroll
     for (int i = 0; i < BLOCK_N / 32; ++i) {
         const int kk = half * (BLOCK_N / 32) + i;
         const uint64_t off = static_cast<uint64_t>((kk * 16 * 128) >> 4);
-        mma_ts(d_tmem, p_tmem + kk * 8, b0 + off, idesc, (i > 0) ? 1u : acc_first);
+        mma_ts(d_tmem, p_tmem + kk * 8, b0 + off, idesc, (i > 0) ? 1u : acc_first, leader);
     }
 }
 
@@ -322,28 +329,29 @@ __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
 }
 
 __device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate) {
+                                          uint32_t idesc, uint32_t accumulate, uint32_t leader) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+        "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 e, %5, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(leader));
 }
 
 __device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate) {
+                                          uint32_t idesc, uint32_t accumulate, uint32_t leader) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
+        "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 e, %5, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(leader));
 }
 
 /* S = Q K^T with e4m3 Q and K, d = 128 (a row is one 128-byte swizzle atom):
  * 4 MMAs with K = 32, each starting 32 bytes further. */
-__device__ __forceinline__ void issue_qk_f8(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc) {
+__device__ __forceinline__ void issue_qk_f8(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc,
+                                            uint32_t leader) {
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
         const uint64_t off = static_cast<uint64_t>((kk * 32) >> 4);
-        mma_ss_f8(d_tmem, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
+        mma_ss_f8(d_tmem, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u, leader);
     }
 }
 
@@ -352,26 +360,29 @@ __device__ __forceinline__ void issue_qk_f8(uint32_t d_tmem, uint64_t a0, uint64
  * describes V^T (d rows, keys contiguous: K-major), 32 keys = 32 bytes further
  * per k-step. */
 __device__ __forceinline__ void issue_pv_half_f8(uint32_t d_tmem, uint32_t p_tmem, uint64_t b0,
-                                                 uint32_t idesc, uint32_t acc_first, int half) {
+                                                 uint32_t idesc, uint32_t acc_first, int half,
+                                                 uint32_t leader) {
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
         const int kk = half * 2 + i;
         mma_ts_f8(d_tmem, p_tmem + kk * 8, b0 + static_cast<uint64_t>((kk * 32) >> 4), idesc,
-                  (i > 0) ? 1u : acc_first);
+                  (i > 0) ? 1u : acc_first, leader);
     }
 }
 
 template <int D, bool FP8>
-__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc) {
-    if constexpr (FP8) issue_qk_f8(d_tmem, a0, b0, idesc);
-    else issue_qk<D>(d_tmem, a0, b0, idesc);
+__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc,
+                                        uint32_t leader) {
+    if constexpr (FP8) issue_qk_f8(d_tmem, a0, b0, idesc, leader);
+    else issue_qk<D>(d_tmem, a0, b0, idesc, leader);
 }
 
 template <bool FP8>
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t b0,
-                                         uint32_t idesc, uint32_t acc_first, int half) {
-    if constexpr (FP8) issue_pv_half_f8(d_tmem, p_tmem, b0, idesc, acc_first, half);
-    else issue_pv_half(d_tmem, p_tmem, b0, idesc, acc_first, half);
+                                         uint32_t idesc, uint32_t acc_first, int half,
+                                         uint32_t leader) {
+    if constexpr (FP8) issue_pv_half_f8(d_tmem, p_tmem, b0, idesc, acc_first, half, leader);
+    else issue_pv_half(d_tmem, p_tmem, b0, idesc, acc_first, half, leader);
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -445,12 +456,14 @@ __device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& p0, fl
 }
 
 /* Which column pairs of a score row take the polynomial (bit k%8 of the mask
- * for pair k); the rest use the MUFU ex2.  3 of 8 pairs balances the MUFU and
- * FMA pipes for a 128-column block. */
-#ifndef ATTN_EXP2_POLY_MASK
-#define ATTN_EXP2_POLY_MASK 0x00u
-#endif
-constexpr uint32_t EXP2_POLY_MASK = ATTN_EXP2_POLY_MASK;
+ * for pair k); the rest use the MUFU ex2.  Measured per head dimension: at
+ * d = 64 (half the tensor work per exponential of d = 128) 2 of 8 pairs on the
+ * FMA pipe was fastest; at d = 128 and for e4m3 every fraction tried was
+ * slower than none. */
+template <int D, bool FP8>
+__device__ __forceinline__ constexpr uint32_t exp2_poly_mask() {
+    return (D == 64 && !FP8) ? 0x11u : 0x00u;
+}
 
 /* Two fp32 -> one bf16x2 word, round to nearest even; `lo` in bits 0-15. */
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -519,6 +532,29 @@ __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t* v) {
           "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
           "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
           "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+/* tcgen05.ld of 64 consecutive 32-bit columns of this thread's TMEM lane, with
+ * the wait in the same asm statement. */
+__device__ __forceinline__ void tmem_ld64_wait(uint32_t taddr, uint32_t* v) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {"
+        "%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+        "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+        "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63"
+        "}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31]),
+          "=r"(v[32]), "=r"(v[33]), "=r"(v[34]), "=r"(v[35]), "=r"(v[36]), "=r"(v[37]), "=r"(v[38]), "=r"(v[39]),
+          "=r"(v[40]), "=r"(v[41]), "=r"(v[42]), "=r"(v[43]), "=r"(v[44]), "=r"(v[45]), "=r"(v[46]), "=r"(v[47]),
+          "=r"(v[48]), "=r"(v[49]), "=r"(v[50]), "=r"(v[51]), "=r"(v[52]), "=r"(v[53]), "=r"(v[54]), "=r"(v[55]),
+          "=r"(v[56]), "=r"(v[57]), "=r"(v[58]), "=r"(v[59]), "=r"(v[60]), "=r"(v[61]), "=r"(v[62]), "=r"(v[63])
         : "r"(taddr)
         : "memory");
 }
@@ -796,14 +832,20 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     } else if (warp == MMA_WARP) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(OTHER_REGS) : "memory");
         /* ---------------- MMA issuer ----------------
-         * Tensor-core order per K/V block j, one thread:
+         * Tensor-core order per K/V block j (one issuing thread):
          *   P0_j V_j, S0_{j+1}, P1_j V_j, S1_{j+1}
          * so each tile's softmax of block j+1 overlaps the other tile's GEMMs.
          * S_t(j+1) overwrites the TMEM columns that hold P_t(j); the tensor
          * core runs one thread's MMAs in order, so P_t(j) V_j reads P first.
          * Waits on TMA barriers need no tcgen05 fence (no tcgen05 op precedes
          * their arrival); waits on softmax barriers do. */
-        if (lane == 0) {
+        {
+            // all 32 lanes run the loop (the descriptor arithmetic stays warp-uniform);
+            // lane 0 issues every MMA and commit
+            const uint32_t ld = lane == 0 ? 1u : 0u;
+            auto wait = [&](uint32_t bar, uint32_t parity) {
+                return __all_sync(0xffffffffu, mbar_wait_inl(bar, parity, abort_flag, wlim));
+            };
             constexpr uint32_t IDESC_S = FP8 ? idesc_e4m3(BLOCK_M, BLOCK_N)
                                              : idesc_bf16(BLOCK_M, BLOCK_N, false);
             constexpr uint32_t IDESC_PV = FP8 ? idesc_e4m3(BLOCK_M, D) : idesc_bf16(BLOCK_M, D, true);
@@ -830,15 +872,15 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                 if (got == 0) continue;
                 const int n0 = u.n[0], n1 = u.n[1];
                 const int nmax = n0 > n1 ? n0 : n1;
-                if (!mbar_wait_inl(bar_q_full, local & 1, abort_flag, wlim)) { aborted = true; break; }
+                if (!wait(bar_q_full, local & 1)) { aborted = true; break; }
                 // block 0: S0_0, S1_0
                 {
                     const uint32_t st = it % NSTAGE;
-                    if (!mbar_wait_inl(bar_kv_full(st), (it / NSTAGE) & 1u, abort_flag, wlim)) { aborted = true; break; }
+                    if (!wait(bar_kv_full(st), (it / NSTAGE) & 1u)) { aborted = true; break; }
                     const uint64_t kd = kd_base + 2 * st * SLOT_STEP;
-                    if (n0 > 0) { issue_s<D, FP8>(ts0, qd0, kd, IDESC_S); mma_commit(bs0); }
-                    if (n1 > 0) { issue_s<D, FP8>(ts1, qd1, kd, IDESC_S); mma_commit(bs1); }
-                    if (nmax == 1) mma_commit(bar_q_empty);
+                    if (n0 > 0) { issue_s<D, FP8>(ts0, qd0, kd, IDESC_S, ld); mma_commit(bs0, ld); }
+                    if (n1 > 0) { issue_s<D, FP8>(ts1, qd1, kd, IDESC_S, ld); mma_commit(bs1, ld); }
+                    if (nmax == 1) mma_commit(bar_q_empty, ld);
                 }
                 for (int j = 0; j < nmax; ++j) {
                     const uint32_t st = it % NSTAGE;                 // stage of block j
@@ -848,40 +890,40 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const uint32_t nx = it + 1;                      // ring position of block j+1
                     const uint64_t kd = kd_base + 2 * (nx % NSTAGE) * SLOT_STEP;
                     if (j < n0) {
-                        if (!mbar_wait_inl(bh0, pr0 & 1u, abort_flag, wlim)) { aborted = true; break; }
+                        if (!wait(bh0, pr0 & 1u)) { aborted = true; break; }
                         tc_fence_after();
-                        issue_pv<FP8>(to0, ts0, vd, IDESC_PV, acc, 0);
-                        if (!mbar_wait_inl(bp0, pr0 & 1u, abort_flag, wlim)) { aborted = true; break; }
+                        issue_pv<FP8>(to0, ts0, vd, IDESC_PV, acc, 0, ld);
+                        if (!wait(bp0, pr0 & 1u)) { aborted = true; break; }
                         ++pr0;
                         tc_fence_after();
-                        issue_pv<FP8>(to0, ts0, vd, IDESC_PV, 1u, 1);
-                        if (j == n0 - 1) mma_commit(bo0);
+                        issue_pv<FP8>(to0, ts0, vd, IDESC_PV, 1u, 1, ld);
+                        if (j == n0 - 1) mma_commit(bo0, ld);
                     }
                     if (has_next &&
-                        !mbar_wait_inl(bar_kv_full(nx % NSTAGE), (nx / NSTAGE) & 1u, abort_flag, wlim)) {
+                        !wait(bar_kv_full(nx % NSTAGE), (nx / NSTAGE) & 1u)) {
                         aborted = true;
                         break;
                     }
-                    if (j + 1 < n0) { issue_s<D, FP8>(ts0, qd0, kd, IDESC_S); mma_commit(bs0); }
+                    if (j + 1 < n0) { issue_s<D, FP8>(ts0, qd0, kd, IDESC_S, ld); mma_commit(bs0, ld); }
                     if (j < n1) {
-                        if (!mbar_wait_inl(bh1, pr1 & 1u, abort_flag, wlim)) { aborted = true; break; }
+                        if (!wait(bh1, pr1 & 1u)) { aborted = true; break; }
                         tc_fence_after();
-                        issue_pv<FP8>(to1, ts1, vd, IDESC_PV, acc, 0);
-                        if (!mbar_wait_inl(bp1, pr1 & 1u, abort_flag, wlim)) { aborted = true; break; }
+                        issue_pv<FP8>(to1, ts1, vd, IDESC_PV, acc, 0, ld);
+                        if (!wait(bp1, pr1 & 1u)) { aborted = true; break; }
                         ++pr1;
                         tc_fence_after();
-                        issue_pv<FP8>(to1, ts1, vd, IDESC_PV, 1u, 1);
-                        if (j == n1 - 1) mma_commit(bo1);
+                        issue_pv<FP8>(to1, ts1, vd, IDESC_PV, 1u, 1, ld);
+                        if (j == n1 - 1) mma_commit(bo1, ld);
                     }
-                    mma_commit(bar_kv_empty(st));                    // K_j and V_j read
+                    mma_commit(bar_kv_empty(st), ld);                    // K_j and V_j read
                     ++it;
-                    if (j + 1 < n1) { issue_s<D, FP8>(ts1, qd1, kd, IDESC_S); mma_commit(bs1); }
-                    if (j + 1 == nmax - 1) mma_commit(bar_q_empty);  // last S of the unit issued
+                    if (j + 1 < n1) { issue_s<D, FP8>(ts1, qd1, kd, IDESC_S, ld); mma_commit(bs1, ld); }
+                    if (j + 1 == nmax - 1) mma_commit(bar_q_empty, ld);  // last S of the unit issued
                 }
                 ++local;
             }
             /* all MMAs this thread issued have completed once this phase lands */
-            mma_commit(bar_drain);
+            mma_commit(bar_drain, ld);
             mbar_drain_wait_inl(bar_drain, 0, wlim);
         }
         __syncwarp();
@@ -975,7 +1017,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                         float x0, x1;
                         f2unpack(ffma2(f2pack(s[cc], s[cc + 1]), c2, nm2), x0, x1);
                         float p0, p1;
-                        if ((EXP2_POLY_MASK >> ((qtr * (BLOCK_N / 8) + k) & 7)) & 1u) {
+                        if ((exp2_poly_mask<D, FP8>() >> ((qtr * (BLOCK_N / 8) + k) & 7)) & 1u) {
                             exp2_poly_pair(x0, x1, p0, p1);
                         } else {
                             p0 = ex2(x0);

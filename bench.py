@@ -483,7 +483,7 @@ def run_cuda(args, w):
             "e2e": {"value": total_flops / (e2e_max * 1e-3) / 1e12 if e2e_max else None,
                     "unit": UNIT, "ms_per_step": e2e_max,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "path": "attn_fwd_host (pinned host buffers, copies + kernel on one stream)"},
+                    "path": "attn_fwd_host (pinned host buffers; above 32 MB the copies in, kernels and copies out of up to 8 chunks of heads overlap on helper streams)"},
             "gpu_launches": launches,
             "clocks": clocks,
         }

@@ -15,7 +15,8 @@
  * bwd_pre_kernel   D_i and LSE_i * log2(e) into row-padded workspace arrays (the
  *                  host zeroes the fp32 dQ accumulator before it).
  * bwd_main_kernel  one CTA per (head, 128-row K/V block j), looping over the Q
- *                  blocks i that see block j.  K_j and V_j stay in shared memory;
+ *                  blocks i that see block j; CTAs start longest first within
+ *                  groups of heads.  K_j and V_j stay in shared memory;
  *                  Q_i and dO_i stream through a 2-stage TMA ring.  Per i, on
  *                  the tensor cores (TMEM accumulators):
  *                      S^T  = K_j Q_i^T   -> TMEM A      dP^T = V_j dO_i^T -> TMEM B
@@ -44,6 +45,7 @@
  * halves, staged in the same layout in shared memory.
  */
 
+constexpr int BWD_HEAD_GROUP = 8;   // heads per group of the grid order (bwd_main_kernel)
 constexpr int BWD_THREADS = 512;    // warps 0-7 P, dS, epilogue; 8 TMA; 9 MMA; 12-15 dQ readout
 constexpr int BWD_COMPUTE = 256;
 constexpr int BWD_LOAD_WARP = 8;
@@ -218,7 +220,19 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     volatile uint32_t* const abort_flag = reinterpret_cast<volatile uint32_t*>(base_ptr + C::MISC_OFF + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t wlim = p.wait_limit_ns;
-    const int jb = blockIdx.x, bh = blockIdx.y;
+    // Grid order: groups of BWD_HEAD_GROUP heads, and within a group every head's
+    // K/V block 0 first, then block 1, ...  The hardware starts CTAs in index
+    // order, so for causal masks (block j has nblk - j Q blocks) the longest
+    // CTAs start first and the end of the launch is made of short ones; a group's
+    // Q, dO, K, V stay within L2 while its CTAs run.
+    int jb, bh;
+    {
+        const int per_group = BWD_HEAD_GROUP * p.nblk;
+        const int g = blockIdx.x / per_group, r = blockIdx.x - g * per_group;
+        const int heads = min(BWD_HEAD_GROUP, p.BH - g * BWD_HEAD_GROUP);
+        jb = r / heads;
+        bh = g * BWD_HEAD_GROUP + (r - jb * heads);
+    }
     const int ib0 = CAUSAL ? jb : 0;
     const int nq = p.nblk - ib0;                 // Q blocks that see this K/V block
 

@@ -1139,6 +1139,9 @@ struct DeviceInfo {
     bool dec_set[2] = {};            // decode stream kernels: D == 128
     bool std_set[2] = {};            // standard-path GEMM kernels: D == 128
     void* scratch = nullptr;         // device address of the no-alloc decode buffer
+    bool host_ready = false;         // helper streams and events of attn_fwd_host below
+    cudaStream_t host_streams[3] = {};   // copies in, kernels, copies out
+    cudaEvent_t host_events[4] = {};     // start, chunk copied in, chunk computed, done
 };
 
 std::mutex g_mutex;
@@ -1224,6 +1227,7 @@ int device_info(int* dev_out, DeviceInfo** info_out) {
         for (int i = 0; i < 4; ++i) di.bwd_set[i] = false;
         for (int i = 0; i < 2; ++i) di.dec_set[i] = di.std_set[i] = false;
         di.scratch = nullptr;
+        di.host_ready = false;   // streams and events of another context are not used here
         di.ctx_id = id;
         di.ctx_known = true;
     }
@@ -1658,7 +1662,7 @@ int bwd_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     bwd_pre_kernel<D><<<static_cast<unsigned>((prows + 7) / 8), 256, 0, stream>>>(
         o, dout, lse, const_cast<float*>(prm.Dp), const_cast<float*>(prm.lse2), prm.N, prm.Np,
         prm.BH);
-    kern<<<dim3(prm.nblk, prm.BH), BWD_THREADS, SMEM, stream>>>(mq, mk, mv, mdo, prm);
+    kern<<<static_cast<unsigned>(prm.nblk * prm.BH), BWD_THREADS, SMEM, stream>>>(mq, mk, mv, mdo, prm);
     bwd_post_kernel<D><<<static_cast<unsigned>(prm.BH * prm.nblk), BLOCK_M, 0, stream>>>(
         prm.dq_acc, prm.dq, prm.N, prm.nblk);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
@@ -1840,28 +1844,87 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
         workspace_bytes < attn_fwd_host_workspace_bytes(B, H, N, d))
         return ATTN_ERR_WORKSPACE;
-    const size_t tbytes = static_cast<size_t>(B * H * N * d) * 2;
-    const size_t lbytes = static_cast<size_t>(B * H * N) * 4;
+    const int64_t BH = B * H;
+    const size_t tbytes = static_cast<size_t>(BH * N * d) * 2;
+    const size_t lbytes = static_cast<size_t>(BH * N) * 4;
     char* ws = static_cast<char*>(workspace);
-    void* dq = ws;
-    void* dk = ws + align256(tbytes);
-    void* dv = ws + 2 * align256(tbytes);
-    void* dout = ws + 3 * align256(tbytes);
-    float* dl = reinterpret_cast<float*>(ws + 4 * align256(tbytes));
+    char* dq = ws;
+    char* dk = ws + align256(tbytes);
+    char* dv = ws + 2 * align256(tbytes);
+    char* dout = ws + 3 * align256(tbytes);
+    char* dl = ws + 4 * align256(tbytes);
+    const char* hq = static_cast<const char*>(q);
+    const char* hk = static_cast<const char*>(k);
+    const char* hv = static_cast<const char*>(v);
+    char* ho = static_cast<char*>(o);
+    char* hl = reinterpret_cast<char*>(lse);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (cudaMemcpyAsync(dq, q, tbytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(dk, k, tbytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(dv, v, tbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
-        cudaGetLastError();
-        return ATTN_ERR_CUDA;
+    auto fail = [] { cudaGetLastError(); return ATTN_ERR_CUDA; };
+
+    /* Heads are independent, so the copies and the kernel are pipelined over
+     * chunks of heads: chunk c's kernel and copy back run while chunk c+1 is
+     * copied in (copies in and out use separate engines).  Small problems take
+     * one chunk. */
+    constexpr size_t MIN_PIPELINED_BYTES = size_t(32) << 20;
+    const int64_t nchunks = (tbytes * 3 < MIN_PIPELINED_BYTES) ? 1 : (BH < 8 ? BH : 8);
+    if (nchunks <= 1) {
+        if (cudaMemcpyAsync(dq, q, tbytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(dk, k, tbytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(dv, v, tbytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return fail();
+        if ((st = attn_fwd(dq, dk, dv, dout, reinterpret_cast<float*>(dl), B, H, N, d, causal,
+                           scale, stream)) != ATTN_OK)
+            return st;
+        if (cudaMemcpyAsync(o, dout, tbytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+            cudaMemcpyAsync(lse, dl, lbytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+            return fail();
+        return ATTN_OK;
     }
-    if ((st = attn_fwd(dq, dk, dv, dout, dl, B, H, N, d, causal, scale, stream)) != ATTN_OK)
-        return st;
-    if (cudaMemcpyAsync(o, dout, tbytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaMemcpyAsync(lse, dl, lbytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
-        cudaGetLastError();
-        return ATTN_ERR_CUDA;
+    int dev = 0;
+    DeviceInfo* di = nullptr;
+    if ((st = device_info(&dev, &di)) != ATTN_OK) return st;
+    // one enqueue sequence at a time per device: the helper streams and events are shared
+    static std::mutex host_mutex;
+    std::lock_guard<std::mutex> lock(host_mutex);
+    {
+        std::lock_guard<std::mutex> dlock(g_mutex);
+        if (!di->host_ready) {
+            for (auto& hs : di->host_streams)
+                if (cudaStreamCreateWithFlags(&hs, cudaStreamNonBlocking) != cudaSuccess) return fail();
+            for (auto& ev : di->host_events)
+                if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return fail();
+            di->host_ready = true;
+        }
     }
+    cudaStream_t s_in = di->host_streams[0], s_k = di->host_streams[1], s_out = di->host_streams[2];
+    cudaEvent_t ev_start = di->host_events[0], ev_in = di->host_events[1];
+    cudaEvent_t ev_k = di->host_events[2], ev_done = di->host_events[3];
+    // everything starts after the work already on the caller's stream
+    if (cudaEventRecord(ev_start, s) != cudaSuccess || cudaStreamWaitEvent(s_in, ev_start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(s_k, ev_start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(s_out, ev_start, 0) != cudaSuccess)
+        return fail();
+    const int64_t per = (BH + nchunks - 1) / nchunks;
+    for (int64_t h0 = 0; h0 < BH; h0 += per) {
+        const int64_t hn = (BH - h0 < per) ? BH - h0 : per;
+        const size_t to = static_cast<size_t>(h0 * N * d) * 2, tn = static_cast<size_t>(hn * N * d) * 2;
+        const size_t lo = static_cast<size_t>(h0 * N) * 4, ln = static_cast<size_t>(hn * N) * 4;
+        if (cudaMemcpyAsync(dq + to, hq + to, tn, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+            cudaMemcpyAsync(dk + to, hk + to, tn, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+            cudaMemcpyAsync(dv + to, hv + to, tn, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+            cudaEventRecord(ev_in, s_in) != cudaSuccess || cudaStreamWaitEvent(s_k, ev_in, 0) != cudaSuccess)
+            return fail();
+        if ((st = attn_fwd(dq + to, dk + to, dv + to, dout + to, reinterpret_cast<float*>(dl + lo), 1, hn,
+                           N, d, causal, scale, s_k)) != ATTN_OK)
+            return st;
+        if (cudaEventRecord(ev_k, s_k) != cudaSuccess || cudaStreamWaitEvent(s_out, ev_k, 0) != cudaSuccess ||
+            cudaMemcpyAsync(ho + to, dout + to, tn, cudaMemcpyDeviceToHost, s_out) != cudaSuccess ||
+            cudaMemcpyAsync(hl + lo, dl + lo, ln, cudaMemcpyDeviceToHost, s_out) != cudaSuccess)
+            return fail();
+    }
+    // the caller's stream continues once the last copy back has finished
+    if (cudaEventRecord(ev_done, s_out) != cudaSuccess || cudaStreamWaitEvent(s, ev_done, 0) != cudaSuccess)
+        return fail();
     return ATTN_OK;
 }
 

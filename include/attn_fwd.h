@@ -81,13 +81,19 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 size_t attn_fwd_host_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
 
 /*
- * attn_fwd_host -- the same operation on HOST buffers.  Enqueues on `stream`:
- * three host-to-device copies of q, k, v into `workspace` (device memory of at
- * least attn_fwd_host_workspace_bytes), the attn_fwd kernel, and two
- * device-to-host copies into o and lse.  Host buffers should be page-locked
- * for the copies to be asynchronous.  The caller synchronises the stream
- * before reading o and lse.  Same shapes, layouts and error codes as attn_fwd;
- * the host pointers need no alignment.
+ * attn_fwd_host -- the same operation on HOST buffers: q, k, v are copied into
+ * `workspace` (device memory of at least attn_fwd_host_workspace_bytes), the
+ * kernel runs there, and O and LSE are copied back into o and lse.  Heads are
+ * independent, so above 32 MB of inputs the work is pipelined over up to 8
+ * chunks of heads: the copies in, the kernels and the copies back of
+ * successive chunks overlap on three helper streams that the library creates
+ * on the first such call per device and CUDA context (with four events; the
+ * calls of one process enqueue their work one at a time).  All of it starts after the work
+ * already on `stream`, and `stream` waits for all of it, so synchronising
+ * `stream` covers the call; smaller problems use `stream` alone.  Host buffers
+ * should be page-locked for the copies to be asynchronous.  The caller
+ * synchronises the stream before reading o and lse.  Same shapes, layouts and
+ * error codes as attn_fwd; the host pointers need no alignment.
  */
 int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
                   int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,

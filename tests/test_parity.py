@@ -192,6 +192,23 @@ def test_host_entry_point_matches_device(attn):
     assert torch.equal(o_h, o_d) and torch.equal(l_h, l_d)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_host_entry_point_pipelined_matches_device(attn, causal):
+    """Above 32 MB of inputs the host entry point pipelines the copies and the
+    kernel over chunks of heads (11 heads: chunks of 2, 2, 2, 2, 2, 1); every
+    head's result is computed as in one call, so the outputs are identical."""
+    q, k, v = inputs.make_qkv(1, 11, 4500, 128, seed=17)
+    o_d, l_d = _run(attn, q, k, v, causal=causal)
+    qp, kp, vp = (t.pin_memory() for t in (q, k, v))
+    o_h, l_h = attn.attn_fwd_host(qp, kp, vp, causal=causal)
+    assert attn.device_status(reset=True) == 0
+    assert torch.equal(o_h, o_d) and torch.equal(l_h, l_d)
+    # a second call through the same helper streams, on a user stream
+    s = torch.cuda.Stream()
+    o_h2, l_h2 = attn.attn_fwd_host(qp, kp, vp, causal=causal, stream=s)
+    assert torch.equal(o_h2, o_d) and torch.equal(l_h2, l_d)
+
+
 def test_no_writes_outside_outputs(attn):
     q, k, v = (t.cuda() for t in inputs.make_qkv(1, 3, 300, 128, seed=16))
     B, H, N, d = q.shape

@@ -299,9 +299,9 @@ def attn_fwd_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_descale
                  scale: float | None = None, out: torch.Tensor | None = None,
                  lse: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
                  stream=None):
-    """The forward pass on e4m3 inputs (torch.float8_e4m3fn [B, H, N, 128] CUDA
-    tensors): the scores use q8*q_descale and k8*k_descale, the values
-    v8*v_descale.  O (bf16) and LSE (fp32) as attn_fwd."""
+    """The forward pass on e4m3 inputs (torch.float8_e4m3fn [B, H, N, d] CUDA
+    tensors, d in {64, 128}): the scores use q8*q_descale and k8*k_descale, the
+    values v8*v_descale.  O (bf16) and LSE (fp32) as attn_fwd."""
     for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
         if not isinstance(t, torch.Tensor):
             raise TypeError(f"{name} must be a torch.Tensor")

@@ -85,8 +85,9 @@ constexpr uint32_t WAIT_MAX_ITERS = 1u << 28;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float LOG2E = 1.4426950408889634f;
 
-/* FP8: e4m3 Q, K, V (d = 128: one 128-byte swizzle atom per row), V read
- * transposed (d rows, keys contiguous) so that every operand is K-major. */
+/* FP8: e4m3 Q, K, V, V read transposed (d rows, keys contiguous) so that every
+ * operand is K-major.  A Q or K row is one 128-byte swizzle atom at d = 128 and
+ * a 64-byte one at d = 64; a V^T row (128 keys of one block) is 128 bytes. */
 template <int D, bool FP8 = false>
 struct Cfg {
     static constexpr int TILE_BYTES = BLOCK_M * D * (FP8 ? 1 : 2);   // 128 rows x D elements
@@ -102,7 +103,8 @@ struct Cfg {
     static constexpr uint32_t S_COL0 = 0, S_COL1 = 128;
     static constexpr uint32_t O_COL0 = 256, O_COL1 = 256 + D;
     static_assert(D == 64 || D == 128, "head dim");
-    static_assert(!FP8 || D == 128, "e4m3 inputs: d = 128 only");
+    // Q and K rows of e4m3 at d = 64 are 64 bytes: 64-byte swizzle (TMA and MMA)
+    static constexpr bool QK_SW64 = FP8 && D == 64;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
@@ -256,6 +258,18 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     return d;
 }
 
+/* The same descriptor with 64-byte swizzle ([61,64) = 4): rows of 64 bytes,
+ * 8-row groups 512 bytes apart. */
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(1) << 16;                      // leading byte offset (unused here)
+    d |= static_cast<uint64_t>((512u >> 4) & 0x3FFFu) << 32;  // stride byte offset
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(4) << 61;
+    return d;
+}
+
 /* Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, dense.
  * Bits: [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format,
  * 15 A major (0 = K), 16 B major (1 = MN), [17,23) N >> 3, [24,29) M >> 4. */
@@ -344,12 +358,13 @@ __device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint
         ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(leader));
 }
 
-/* S = Q K^T with e4m3 Q and K, d = 128 (a row is one 128-byte swizzle atom):
- * 4 MMAs with K = 32, each starting 32 bytes further. */
+/* S = Q K^T with e4m3 Q and K (a row of D bytes is one swizzle atom, 128- or
+ * 64-byte): D / 32 MMAs with K = 32, each starting 32 bytes further. */
+template <int D>
 __device__ __forceinline__ void issue_qk_f8(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc,
                                             uint32_t leader) {
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
+    for (int kk = 0; kk < D / 32; ++kk) {
         const uint64_t off = static_cast<uint64_t>((kk * 32) >> 4);
         mma_ss_f8(d_tmem, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u, leader);
     }
@@ -373,7 +388,7 @@ __device__ __forceinline__ void issue_pv_half_f8(uint32_t d_tmem, uint32_t p_tme
 template <int D, bool FP8>
 __device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc,
                                         uint32_t leader) {
-    if constexpr (FP8) issue_qk_f8(d_tmem, a0, b0, idesc, leader);
+    if constexpr (FP8) issue_qk_f8<D>(d_tmem, a0, b0, idesc, leader);
     else issue_qk<D>(d_tmem, a0, b0, idesc, leader);
 }
 
@@ -852,9 +867,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             constexpr uint64_t SLOT_STEP = TILE >> 4;       // descriptor units per ring slot
             const uint32_t ts0 = tmem + C::S_COL0, ts1 = tmem + C::S_COL1;
             const uint32_t to0 = tmem + C::O_COL0, to1 = tmem + C::O_COL1;
-            const uint64_t qd0 = sdesc_sw128(sQ[0], 16, 1024);
-            const uint64_t qd1 = sdesc_sw128(sQ[1], 16, 1024);
-            const uint64_t kd_base = sdesc_sw128(sRing, 16, 1024);                    // K-major
+            const uint64_t qd0 = C::QK_SW64 ? sdesc_sw64(sQ[0]) : sdesc_sw128(sQ[0], 16, 1024);
+            const uint64_t qd1 = C::QK_SW64 ? sdesc_sw64(sQ[1]) : sdesc_sw128(sQ[1], 16, 1024);
+            const uint64_t kd_base = C::QK_SW64 ? sdesc_sw64(sRing)                   // K-major
+                                                : sdesc_sw128(sRing, 16, 1024);
             const uint64_t vd_base = FP8 ? sdesc_sw128(sRing + TILE, 16, 1024)        // V^T, K-major
                                          : sdesc_sw128(sRing + TILE, CHUNK_BYTES, 1024);  // MN-major
             const uint32_t bs0 = bar_s_full0, bs1 = bar_s_full0 + 8;
@@ -1351,12 +1367,12 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
 /* ------------------------------------------------------------------------ */
 /* e4m3 inputs: V transposed into the workspace, then the same kernel        */
 /* ------------------------------------------------------------------------ */
-/* V [BH, N, 128] e4m3 -> V^T [BH, 128, Np] (Np = N rounded up to 128; keys
- * past N are zero, so masked keys multiply zeros).  One CTA per (head, block
- * of 128 keys).  A thread reads four keys x 16 bytes, transposes the 4 x 4
- * byte blocks in registers and parks 32-bit words (4 keys of one column) in
- * shared memory; the CTA then writes the block's 128 rows of V^T with
- * 16-byte stores. */
+/* V [BH, N, D] e4m3 -> V^T [BH, D, Np] (Np = N rounded up to 128; keys past N
+ * are zero, so masked keys multiply zeros).  One CTA of 2 D threads per (head,
+ * block of 128 keys).  A thread reads four keys x 16 bytes, transposes the
+ * 4 x 4 byte blocks in registers and parks 32-bit words (4 keys of one column)
+ * in shared memory; the CTA then writes the block's D rows of V^T with 16-byte
+ * stores. */
 __device__ __forceinline__ void transpose4x4_bytes(const uint32_t w[4], uint32_t out[4]) {
     // out[c] = byte c of w[0], w[1], w[2], w[3] (w[r] in byte r)
     const uint32_t lo01 = __byte_perm(w[0], w[1], 0x5140), hi01 = __byte_perm(w[0], w[1], 0x7362);
@@ -1367,20 +1383,22 @@ __device__ __forceinline__ void transpose4x4_bytes(const uint32_t w[4], uint32_t
     out[3] = __byte_perm(hi01, hi23, 0x7632);
 }
 
-__global__ void __launch_bounds__(256)
+template <int D>
+__global__ void __launch_bounds__(2 * D)
 fp8_transpose_v_kernel(const uint8_t* __restrict__ v, uint8_t* __restrict__ vt, int N, int Np) {
-    __shared__ uint32_t tw[128][33];          // [column][group of 4 keys], padded row
+    constexpr int C16 = D / 16;               // 16-byte pieces of a V row
+    __shared__ uint32_t tw[D][33];            // [column][group of 4 keys], padded row
     const int kb = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
-    const uint8_t* src = v + (static_cast<int64_t>(bh) * N + static_cast<int64_t>(kb) * 128) * 128;
+    const uint8_t* src = v + (static_cast<int64_t>(bh) * N + static_cast<int64_t>(kb) * 128) * D;
     {
-        const int g = t >> 3, c16 = t & 7;    // keys 4g .. 4g+3, columns 16 c16 .. 16 c16 + 15
+        const int g = t / C16, c16 = t % C16;  // keys 4g .. 4g+3, columns 16 c16 .. 16 c16 + 15
         uint4 rows[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const int key = 4 * g + r;
             rows[r] = make_uint4(0u, 0u, 0u, 0u);
             if (kb * 128 + key < N)
-                rows[r] = *reinterpret_cast<const uint4*>(src + key * 128 + c16 * 16);
+                rows[r] = *reinterpret_cast<const uint4*>(src + key * D + c16 * 16);
         }
 #pragma unroll
         for (int wi = 0; wi < 4; ++wi) {
@@ -1395,33 +1413,35 @@ fp8_transpose_v_kernel(const uint8_t* __restrict__ v, uint8_t* __restrict__ vt, 
         }
     }
     __syncthreads();
-    uint8_t* dst = vt + static_cast<int64_t>(bh) * 128 * Np + static_cast<int64_t>(kb) * 128;
+    uint8_t* dst = vt + static_cast<int64_t>(bh) * D * Np + static_cast<int64_t>(kb) * 128;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int item = t + 256 * i;         // 128 columns x 8 runs of 16 keys
+        const int item = t + 2 * D * i;       // D columns x 8 runs of 16 keys
         const int col = item >> 3, u = item & 7;
         *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(col) * Np + u * 16) =
             make_uint4(tw[col][4 * u], tw[col][4 * u + 1], tw[col][4 * u + 2], tw[col][4 * u + 3]);
     }
 }
 
-/* 3-D map over 8-bit data [BH][rows][inner], box 128 x 128 bytes, 128B swizzle. */
+/* 3-D map over 8-bit data [BH][rows][inner], box box_inner bytes x box_rows
+ * rows: 128-byte swizzle for 128-byte box rows, 64-byte swizzle for 64-byte ones. */
 int encode_map_u8(EncodeTiledFn fn, CUtensorMap* map, const void* ptr, int64_t BH, int64_t rows,
-                  int64_t inner) {
+                  int64_t inner, uint32_t box_inner = 128, uint32_t box_rows = BLOCK_M) {
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
                           static_cast<cuuint64_t>(BH)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows * inner)};
-    cuuint32_t box[3] = {128, BLOCK_M, 1};
+    cuuint32_t box[3] = {box_inner, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    box_inner == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-size_t fp8_ws_bytes(int64_t BH, int64_t N) {
+size_t fp8_ws_bytes(int64_t BH, int64_t N, int64_t d) {
     const int64_t Np = (N + BLOCK_N - 1) / BLOCK_N * BLOCK_N;
-    return static_cast<size_t>(BH) * 128 * Np;
+    return static_cast<size_t>(BH) * d * Np;
 }
 
 int fp8_impl(const void* q, const void* k, const void* v, float q_descale, float k_descale,
@@ -1430,7 +1450,6 @@ int fp8_impl(const void* q, const void* k, const void* v, float q_descale, float
     bool empty = false;
     int st = validate_shape(B, H, N, d, scale, &empty);
     if (st != ATTN_OK) return st;
-    if (d != 128) return ATTN_ERR_HEADDIM;
     if (empty) return ATTN_OK;
     if (B * H > 65535) return ATTN_ERR_SHAPE;
     const float ds[3] = {q_descale, k_descale, v_descale};
@@ -1443,7 +1462,7 @@ int fp8_impl(const void* q, const void* k, const void* v, float q_descale, float
         if (reinterpret_cast<uintptr_t>(ptr) & 15u) return ATTN_ERR_ALIGN;
     }
     const int64_t BH = B * H;
-    const size_t ws_need = fp8_ws_bytes(BH, N);
+    const size_t ws_need = fp8_ws_bytes(BH, N, d);
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < ws_need)
         return ATTN_ERR_WORKSPACE;
     const size_t in_bytes = static_cast<size_t>(BH * N * d);
@@ -1463,14 +1482,21 @@ int fp8_impl(const void* q, const void* k, const void* v, float q_descale, float
     if ((st = get_encode(&enc)) != ATTN_OK) return st;
     const int64_t Np = (N + BLOCK_N - 1) / BLOCK_N * BLOCK_N;
     CUtensorMap mq, mk, mvt;
-    if ((st = encode_map_u8(enc, &mq, q, BH, N, d)) != ATTN_OK) return st;
-    if ((st = encode_map_u8(enc, &mk, k, BH, N, d)) != ATTN_OK) return st;
-    if ((st = encode_map_u8(enc, &mvt, workspace, BH, d, Np)) != ATTN_OK) return st;
+    const uint32_t qk_box = static_cast<uint32_t>(d);   // a Q / K row: 128 or 64 bytes
+    if ((st = encode_map_u8(enc, &mq, q, BH, N, d, qk_box)) != ATTN_OK) return st;
+    if ((st = encode_map_u8(enc, &mk, k, BH, N, d, qk_box)) != ATTN_OK) return st;
+    if ((st = encode_map_u8(enc, &mvt, workspace, BH, d, Np, 128, static_cast<uint32_t>(d))) != ATTN_OK)
+        return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    fp8_transpose_v_kernel<<<dim3(static_cast<unsigned>(Np / BLOCK_N), static_cast<unsigned>(BH)),
-                             256, 0, s>>>(static_cast<const uint8_t*>(v),
-                                          static_cast<uint8_t*>(workspace), static_cast<int>(N),
-                                          static_cast<int>(Np));
+    const dim3 tgrid(static_cast<unsigned>(Np / BLOCK_N), static_cast<unsigned>(BH));
+    if (d == 64)
+        fp8_transpose_v_kernel<64><<<tgrid, 128, 0, s>>>(static_cast<const uint8_t*>(v),
+                                                         static_cast<uint8_t*>(workspace),
+                                                         static_cast<int>(N), static_cast<int>(Np));
+    else
+        fp8_transpose_v_kernel<128><<<tgrid, 256, 0, s>>>(static_cast<const uint8_t*>(v),
+                                                          static_cast<uint8_t*>(workspace),
+                                                          static_cast<int>(N), static_cast<int>(Np));
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
     FwdParams prm;
     prm.o = static_cast<__nv_bfloat16*>(o);
@@ -1484,6 +1510,9 @@ int fp8_impl(const void* q, const void* k, const void* v, float q_descale, float
     prm.wait_limit_ns = WAIT_LIMIT_NS;
     prm.withhold_kv = 0;
     prm.o_scale = v_descale;
+    if (d == 64)
+        return causal ? launch<64, true, true>(mq, mk, mvt, prm, di, s)
+                      : launch<64, false, true>(mq, mk, mvt, prm, di, s);
     return causal ? launch<128, true, true>(mq, mk, mvt, prm, di, s)
                   : launch<128, false, true>(mq, mk, mvt, prm, di, s);
 }
@@ -1785,9 +1814,8 @@ int64_t attn_fwd_schedule(int64_t B, int64_t H, int64_t N, int causal, int grid,
 
 size_t attn_fwd_fp8_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {
     bool empty = false;
-    if (validate_shape(B, H, N, d, 1.0f, &empty) != ATTN_OK || empty || d != 128 || B * H > 65535)
-        return 0;
-    return fp8_ws_bytes(B * H, N);
+    if (validate_shape(B, H, N, d, 1.0f, &empty) != ATTN_OK || empty || B * H > 65535) return 0;
+    return fp8_ws_bytes(B * H, N, d);
 }
 
 int attn_fwd_fp8(const void* q, const void* k, const void* v, float q_descale, float k_descale,

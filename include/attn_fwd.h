@@ -161,8 +161,8 @@ int attn_standard(const void* q, const void* k, const void* v, void* o, float* l
 
 /*
  * attn_fwd_fp8_workspace_bytes -- device workspace attn_fwd_fp8 needs: V
- * transposed, B*H*128*Np bytes (Np = N rounded up to 128).  0 for invalid or
- * empty shapes and for d != 128.
+ * transposed, B*H*d*Np bytes (Np = N rounded up to 128).  0 for invalid or
+ * empty shapes (d must be 64 or 128).
  */
 size_t attn_fwd_fp8_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
 
@@ -180,7 +180,7 @@ size_t attn_fwd_fp8_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
  *             caller-owned, contents ignored on entry; it must not overlap the
  *             inputs or outputs (ATTN_ERR_OVERLAP), and calls that overlap on
  *             the GPU must not share it.
- * d must be 128 (ATTN_ERR_HEADDIM otherwise); B*H <= 65535.  Two kernels are
+ * d is 64 or 128 (ATTN_ERR_HEADDIM otherwise); B*H <= 65535.  Two kernels are
  * enqueued on `stream` (V transposed into the workspace, then the forward
  * kernel).  Otherwise the conventions of attn_fwd.  Rounding P to e4m3 (3
  * mantissa bits) makes |dO| up to 2^-4 * max_j |v_j| per element of O.

@@ -92,8 +92,9 @@ def test_binding_rejects_wrong_inputs():
     q8 = q.to(torch.float8_e4m3fn)
     with pytest.raises(ValueError):          # CPU tensors
         m.attn_fwd_fp8(q8, q8, q8)
-    assert m.fp8_workspace_bytes(1, 1, 4, 64) == 0
+    assert m.fp8_workspace_bytes(1, 1, 4, 96) == 0
     assert m.fp8_workspace_bytes(2, 3, 300, 128) == 2 * 3 * 128 * 384
+    assert m.fp8_workspace_bytes(2, 3, 300, 64) == 2 * 3 * 64 * 384     # V^T [BH][d][Np]
 
 
 # ---------------------------------------------------------------------------
@@ -121,23 +122,24 @@ EDGE_N = [1, 2, 127, 128, 129, 255, 256, 257, 300, 385, 1000]
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", EDGE_N)
-def test_edge_shapes(attn, N, causal):
-    d = 128
+def test_edge_shapes(attn, N, causal, d):
     q8, k8, v8 = inputs.make_qkv_e4m3(1, 2, N, d, seed=300 + N)
     scale = 1.0 / math.sqrt(d)
     o, lse = _run(attn, q8, k8, v8, (1.0, 1.0, 1.0), causal, scale)
     q, k, v = (_deq(t, 1.0) for t in (q8, k8, v8))
-    _check(o, lse, q, k, v, causal, scale, [0, 1], np.arange(N), f"N={N} causal={causal}")
+    _check(o, lse, q, k, v, causal, scale, [0, 1], np.arange(N), f"N={N} causal={causal} d={d}")
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
-def test_descales(attn, causal):
+def test_descales(attn, causal, d):
     """Inputs with amplitude 40 (beyond e4m3's 448 after q.k growth is fine, but
     the values themselves need the descale): q8 = x / 4, k8 = x / 8, v8 = x / 16."""
-    N, d = 700, 128
+    N = 700
     ds = (4.0, 8.0, 16.0)
     q8, _, _ = inputs.make_qkv_e4m3(1, 3, N, d, seed=41, amplitude=40.0, descale=ds[0])
     _, k8, _ = inputs.make_qkv_e4m3(1, 3, N, d, seed=41, amplitude=40.0, descale=ds[1])
@@ -159,10 +161,11 @@ def test_many_heads_more_units_than_sms(attn):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("name", ["b4h16_n8192_d128_causal", "b1h16_n32768_d128_causal_peaked"])
+@pytest.mark.parametrize("name", ["b4h16_n8192_d128_causal", "b1h16_n32768_d128_causal_peaked",
+                                  "b8h16_n2048_d64", "b32h32_n512_d64"])
 def test_workload_sampled_rows(attn, name):
-    """Full-size d = 128 workloads, in the launch configuration bench.py times,
-    checked on sampled rows of sampled heads."""
+    """Full-size workloads (d = 128 and d = 64), in the launch configuration
+    bench.py times, checked on sampled rows of sampled heads."""
     w = inputs.WORKLOADS[name]
     q8, k8, v8 = inputs.make_qkv_e4m3(w.B, w.H, w.N, w.d, seed=w.seed)
     o, lse = _run(attn, q8, k8, v8, (1.0, 1.0, 1.0), w.causal, w.scale)
@@ -174,10 +177,11 @@ def test_workload_sampled_rows(attn, name):
 
 
 @pytest.mark.gpu
-def test_close_to_the_bf16_kernel_on_the_same_values(attn):
+@pytest.mark.parametrize("d", [64, 128])
+def test_close_to_the_bf16_kernel_on_the_same_values(attn, d):
     """e4m3 values are exact in bf16: the bf16 kernel sees the same inputs, and
     the two outputs differ only by the rounding of P (bf16 vs e4m3)."""
-    N, d = 1024, 128
+    N = 1024
     q8, k8, v8 = inputs.make_qkv_e4m3(1, 4, N, d, seed=9)
     scale = 1.0 / math.sqrt(d)
     o8, l8 = _run(attn, q8, k8, v8, (1.0, 1.0, 1.0), True, scale)
@@ -201,7 +205,7 @@ def test_error_codes(attn):
     p = q8.data_ptr()
     args = lambda d, dsc, wsb: (p, p, p, dsc, 1.0, 1.0, o.data_ptr(), lse.data_ptr(), 1, 1, 128, d,
                                 0, 0.1, ws.data_ptr(), wsb, None)
-    assert lib.attn_fwd_fp8(*args(64, 1.0, ws.numel())) == ATTN_ERR_HEADDIM
+    assert lib.attn_fwd_fp8(*args(96, 1.0, ws.numel())) == ATTN_ERR_HEADDIM
     assert lib.attn_fwd_fp8(*args(128, 0.0, ws.numel())) == ATTN_ERR_SCALE
     assert lib.attn_fwd_fp8(*args(128, float("nan"), ws.numel())) == ATTN_ERR_SCALE
     assert lib.attn_fwd_fp8(*args(128, 1.0, ws.numel() - 1)) == ATTN_ERR_WORKSPACE

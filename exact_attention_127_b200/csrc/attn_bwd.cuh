@@ -457,7 +457,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const float* dvec = p.Dp + row0;
             // on the diagonal block key r is masked for the queries before it:
             // column ch * 32 + e of this half is masked when it is < mask_lim
-            const int mask_lim = (CAUSAL && ib == jb) ? r - 64 * h : 0;
+            const bool diag = CAUSAL && ib == jb;
+            const int mask_lim = diag ? r - 64 * h : 0;
             float pf[64];
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) {
@@ -474,10 +475,11 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     f2unpack(ffma2(f2pack(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])), c2,
                                    f2pack(-l4.z, -l4.w)), x[2], x[3]);
 #pragma unroll
-                    for (int hh = 0; hh < 4; ++hh) {
-                        float pv = ex2(x[hh]);
-                        if (ch * 32 + e + hh < mask_lim) pv = 0.0f;
-                        pf[ch * 32 + e + hh] = pv;
+                    for (int hh = 0; hh < 4; ++hh) pf[ch * 32 + e + hh] = ex2(x[hh]);
+                    if (diag) {   // warp-uniform: only the diagonal block masks
+#pragma unroll
+                        for (int hh = 0; hh < 4; ++hh)
+                            if (ch * 32 + e + hh < mask_lim) pf[ch * 32 + e + hh] = 0.0f;
                     }
                     pk[e / 2] = pack_bf16(pf[ch * 32 + e], pf[ch * 32 + e + 1]);
                     pk[e / 2 + 1] = pack_bf16(pf[ch * 32 + e + 2], pf[ch * 32 + e + 3]);

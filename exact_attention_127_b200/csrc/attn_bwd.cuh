@@ -85,7 +85,7 @@ struct BwdCfg {
     static constexpr uint32_t DO_OFF = 4 * TILE;                // [2] stages
     static constexpr uint32_t DS_OFF = 6 * TILE;                // 128 x 128 bf16 = 32 KB
     static constexpr uint32_t BAR_OFF = DS_OFF + 32768;
-    static constexpr int NUM_BARS = 15;
+    static constexpr int NUM_BARS = 20;
     static constexpr uint32_t MISC_OFF = BAR_OFF + 8 * NUM_BARS;
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
     // TMEM columns: S^T / P^T, dP^T, the dV and dK accumulators, the dQ partial
@@ -96,6 +96,11 @@ struct BwdCfg {
     // dV_i and the next S^T as soon as P^T is in TMEM, before dS: faster where
     // dQ has columns of its own (D = 64); at D = 128 the later order measured faster
     static constexpr bool EARLY_NEXT_S = !DQ_OVER_DP;
+    // The Q half of a ring stage goes back to the producer as soon as its dQ
+    // reduce has read it (D = 64), or only once the dO half is staged too
+    // (D = 128, where the dQ columns lie under dP^T: stalling the readout warp on
+    // the first reduce would delay their release and with it the next dP^T)
+    static constexpr bool EAGER_Q_FREE = !DQ_OVER_DP;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
@@ -210,12 +215,18 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t sK = base + C::K_OFF, sV = base + C::V_OFF, sDS = base + C::DS_OFF;
     const uint32_t bars = base + C::BAR_OFF;
     const uint32_t bar_kv = bars;
-    auto bar_full = [&](int s) { return bars + 8 + 8u * s; };
+    // Q_i and dO_i of a stage land, and are handed back, separately: the readout
+    // stages the first half of the dQ partial over Q_i and reduce-adds it first,
+    // so the next Q block can load while the second half (over dO_i) is staged
+    auto bar_full_q = [&](int s) { return bars + 8 + 8u * s; };
     auto bar_empty = [&](int s) { return bars + 24 + 8u * s; };
     const uint32_t bar_s = bars + 40, bar_p = bars + 48, bar_pt = bars + 56, bar_dqf = bars + 64;
     const uint32_t bar_dkv = bars + 72, bar_drain = bars + 80, bar_dp = bars + 88;
-    auto bar_free = [&](int s) { return bars + 96 + 8u * s; };   // stage s handed back by the readout
-    const uint32_t bar_rd = bars + 112;                          // the dQ tile is in shared memory
+    auto bar_free_q = [&](int s) { return bars + 96 + 8u * s; };    // Q half of stage s handed back
+    const uint32_t bar_rd_q = bars + 112;                           // first half of the dQ tile staged
+    auto bar_full_do = [&](int s) { return bars + 120 + 8u * s; };
+    auto bar_free_do = [&](int s) { return bars + 136 + 8u * s; };  // dO half of stage s handed back
+    const uint32_t bar_rd_do = bars + 152;                          // second half staged
     uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::MISC_OFF);
     volatile uint32_t* const abort_flag = reinterpret_cast<volatile uint32_t*>(base_ptr + C::MISC_OFF + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -239,11 +250,14 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (threadIdx.x == 0) {
         mbar_init(bar_kv, 1);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(bar_full(s), 1);
+            mbar_init(bar_full_q(s), 1);
+            mbar_init(bar_full_do(s), 1);
             mbar_init(bar_empty(s), 1);
-            mbar_init(bar_free(s), 1);
+            mbar_init(bar_free_q(s), 1);
+            mbar_init(bar_free_do(s), 1);
         }
-        mbar_init(bar_rd, BWD_READERS);
+        mbar_init(bar_rd_q, BWD_READERS);
+        mbar_init(bar_rd_do, BWD_READERS);
         mbar_init(bar_s, 1);
         mbar_init(bar_dp, 1);
         mbar_init(bar_p, BWD_COMPUTE);
@@ -274,26 +288,32 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tma_load_3d(&tm_k, sK + c * CHUNK_BYTES, bar_kv, c * CHUNK_ELEMS, jb * BLOCK_M, bh);
                 tma_load_3d(&tm_v, sV + c * CHUNK_BYTES, bar_kv, c * CHUNK_ELEMS, jb * BLOCK_M, bh);
             }
-            int issued = 0;
+            int issued_q = 0, issued_do = 0;
             for (int it = 0; it < nq; ++it) {
                 const int s = it & 1;
-                if (!mbar_wait_inl(bar_free(s), ((it >> 1) & 1) ^ 1, abort_flag, wlim)) break;
                 const int ib = ib0 + it;
-                mbar_arrive_expect_tx(bar_full(s), 2 * TILE);
-                for (int c = 0; c < C::CHUNKS; ++c) {
-                    tma_load_3d(&tm_q, base + C::Q_OFF + s * TILE + c * CHUNK_BYTES, bar_full(s),
+                if (!mbar_wait_inl(bar_free_q(s), ((it >> 1) & 1) ^ 1, abort_flag, wlim)) break;
+                mbar_arrive_expect_tx(bar_full_q(s), TILE);
+                for (int c = 0; c < C::CHUNKS; ++c)
+                    tma_load_3d(&tm_q, base + C::Q_OFF + s * TILE + c * CHUNK_BYTES, bar_full_q(s),
                                 c * CHUNK_ELEMS, ib * BLOCK_M, bh);
-                    tma_load_3d(&tm_do, base + C::DO_OFF + s * TILE + c * CHUNK_BYTES, bar_full(s),
+                ++issued_q;
+                if (!mbar_wait_inl(bar_free_do(s), ((it >> 1) & 1) ^ 1, abort_flag, wlim)) break;
+                mbar_arrive_expect_tx(bar_full_do(s), TILE);
+                for (int c = 0; c < C::CHUNKS; ++c)
+                    tma_load_3d(&tm_do, base + C::DO_OFF + s * TILE + c * CHUNK_BYTES, bar_full_do(s),
                                 c * CHUNK_ELEMS, ib * BLOCK_M, bh);
-                }
-                ++issued;
+                ++issued_do;
             }
             // every copy this thread issued lands before the CTA can exit
             mbar_drain_wait_inl(bar_kv, 0, wlim);
-            const int back = issued < 2 ? issued : 2;
-            for (int b = 1; b <= back; ++b) {
-                const int it = issued - b;
-                mbar_drain_wait_inl(bar_full(it & 1), (it >> 1) & 1, wlim);
+            for (int b = 1; b <= (issued_q < 2 ? issued_q : 2); ++b) {
+                const int it = issued_q - b;
+                mbar_drain_wait_inl(bar_full_q(it & 1), (it >> 1) & 1, wlim);
+            }
+            for (int b = 1; b <= (issued_do < 2 ? issued_do : 2); ++b) {
+                const int it = issued_do - b;
+                mbar_drain_wait_inl(bar_full_do(it & 1), (it >> 1) & 1, wlim);
             }
         }
         __syncwarp();
@@ -312,7 +332,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint64_t ds_mn = sdesc_sw128(sDS, 16384, 1024);           // dS as MN-major A (dQ)
             const uint64_t ds_k = sdesc_sw128(sDS, 16, 1024);               // dS^T as K-major A (dK)
             bool ok = mbar_wait_inl(bar_kv, 0, abort_flag, wlim);
-            if (ok) ok = mbar_wait_inl(bar_full(0), 0, abort_flag, wlim);
+            if (ok) ok = mbar_wait_inl(bar_full_q(0), 0, abort_flag, wlim);
             if (ok) {
                 tc_fence_after();
                 issue_qk<D>(ta, kd, sdesc_sw128(base + C::Q_OFF, 16, 1024), ID_KQ);  // S^T = K Q^T
@@ -327,6 +347,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (!ok) break;
                     tc_fence_after();
                 }
+                ok = mbar_wait_inl(bar_full_do(s), (it >> 1) & 1, abort_flag, wlim);   // dO_i landed
+                if (!ok) break;
                 issue_qk<D>(tb, vd, sdesc_sw128(sdo, 16, 1024), ID_KQ);         // dP^T = V dO^T
                 mma_commit(bar_dp);
                 const uint64_t do_mn = sdesc_sw128(sdo, CHUNK_BYTES, 1024);
@@ -335,7 +357,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 auto issue_next_s = [&]() -> bool {
                     if (it + 1 >= nq) return true;
                     const int s1 = s ^ 1;
-                    if (!mbar_wait_inl(bar_full(s1), ((it + 1) >> 1) & 1, abort_flag, wlim)) return false;
+                    if (!mbar_wait_inl(bar_full_q(s1), ((it + 1) >> 1) & 1, abort_flag, wlim)) return false;
                     tc_fence_after();
                     issue_qk<D>(ta, kd, sdesc_sw128(base + C::Q_OFF + s1 * TILE, 16, 1024), ID_KQ);
                     mma_commit(bar_s);
@@ -388,10 +410,11 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
          * Once dK_i has read Q_i (so the stage of Q_i and dO_i is free), thread
          * r = query row copies its row of the partial from TMEM into that stage,
          * laid out as the accumulator tile (first half over Q_i, second over
-         * dO_i), and releases the dQ columns.  One thread then adds the tile into
-         * the fp32 accumulator with two TMA bulk reduce-adds and hands the stage
-         * back to the producer once they have read it: no atomics through the
-         * SM's load/store path. */
+         * dO_i), and releases the dQ columns.  One thread adds each half into the
+         * fp32 accumulator with a TMA bulk reduce-add as soon as it is staged, and
+         * hands that half of the stage back to the producer once the reduce has
+         * read it, so the next Q block's load need not wait for the dO half: no
+         * atomics through the SM's load/store path. */
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -403,33 +426,51 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!ok) break;
             tc_fence_after();
             const uint32_t sq = base + C::Q_OFF + s * TILE, sdo = base + C::DO_OFF + s * TILE;
+            float* tile = p.dq_acc + (static_cast<int64_t>(bh) * p.nblk + ib) * (BLOCK_M * D);
+            // half 0 (column groups [0, D/8)) over Q_i, half 1 over dO_i; each half is
+            // reduce-added, and its stage half handed back, as soon as it is staged
 #pragma unroll 1
-            for (int ch = 0; ch < D / 32; ++ch) {
-                uint32_t v[32];
-                tmem_ld32_wait(lane_base + C::DQ_COL + ch * 32, v);
-                if (ch == D / 32 - 1) {          // every column read: release them
-                    tc_fence_before();
-                    mbar_arrive(bar_dqf);
-                }
+            for (int half = 0; half < 2 && ok; ++half) {
+                const uint32_t dst0 = half ? sdo : sq;
+#pragma unroll 1
+                for (int ch = half * (D / 64); ch < (half + 1) * (D / 64); ++ch) {
+                    uint32_t v[32];
+                    tmem_ld32_wait(lane_base + C::DQ_COL + ch * 32, v);
+                    if (ch == D / 32 - 1) {          // every column read: release them
+                        tc_fence_before();
+                        mbar_arrive(bar_dqf);
+                    }
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int g = ch * 8 + e;     // float4 column group of the tile
-                    const uint32_t dst = (g < D / 8 ? sq : sdo) + ((g % (D / 8)) * BLOCK_M + r) * 16;
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[4 * e]),
-                                 "r"(v[4 * e + 1]), "r"(v[4 * e + 2]), "r"(v[4 * e + 3]) : "memory");
+                    for (int e = 0; e < 8; ++e) {
+                        const int g = ch * 8 + e;     // float4 column group of the tile
+                        const uint32_t dst = dst0 + ((g % (D / 8)) * BLOCK_M + r) * 16;
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[4 * e]),
+                                     "r"(v[4 * e + 1]), "r"(v[4 * e + 2]), "r"(v[4 * e + 3]) : "memory");
+                    }
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the TMA
+                const uint32_t bar_rd = half ? bar_rd_do : bar_rd_q;
+                mbar_arrive(bar_rd);
+                if (leader) {
+                    if (!mbar_wait_inl(bar_rd, it & 1, abort_flag, wlim)) { ok = false; break; }
+                    bulk_reduce_add_f32(tile + half * (TILE / 4), dst0, TILE);
+                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                    if (half == 0) {
+                        if constexpr (C::EAGER_Q_FREE) {
+                            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // Q half read
+                            mbar_arrive(bar_free_q(s));
+                        }
+                    } else {
+                        if constexpr (!C::EAGER_Q_FREE) {
+                            asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");   // Q half read
+                            mbar_arrive(bar_free_q(s));
+                        }
+                        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // dO half read
+                        mbar_arrive(bar_free_do(s));
+                    }
                 }
             }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the TMA
-            mbar_arrive(bar_rd);
-            if (leader) {
-                if (!mbar_wait_inl(bar_rd, it & 1, abort_flag, wlim)) break;
-                float* tile = p.dq_acc + (static_cast<int64_t>(bh) * p.nblk + ib) * (BLOCK_M * D);
-                bulk_reduce_add_f32(tile, sq, TILE);
-                bulk_reduce_add_f32(tile + TILE / 4, sdo, TILE);
-                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // the stage is read
-                mbar_arrive(bar_free(s));
-            }
+            if (!ok) break;
         }
         if (leader) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");   // reduces complete
     } else if (warp >= 8) {

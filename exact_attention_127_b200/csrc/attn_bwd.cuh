@@ -81,11 +81,15 @@ struct BwdCfg {
     static constexpr uint32_t TILE = BLOCK_M * D * 2;
     static constexpr int CHUNKS = D / CHUNK_ELEMS;
     static constexpr uint32_t K_OFF = 0, V_OFF = TILE;
-    static constexpr uint32_t Q_OFF = 2 * TILE;                 // [2] stages
-    static constexpr uint32_t DO_OFF = 4 * TILE;                // [2] stages
-    static constexpr uint32_t DS_OFF = 6 * TILE;                // 128 x 128 bf16 = 32 KB
+    // Q_i / dO_i ring: 2 stages at D = 128 (shared memory is full), 4 at D = 64,
+    // where the load of Q block i+2 then need not wait for block i's dQ partial
+    // to leave the stage it is staged in
+    static constexpr int QS = D == 64 ? 4 : 2;
+    static constexpr uint32_t Q_OFF = 2 * TILE;                 // [QS] stages
+    static constexpr uint32_t DO_OFF = Q_OFF + QS * TILE;       // [QS] stages
+    static constexpr uint32_t DS_OFF = DO_OFF + QS * TILE;      // 128 x 128 bf16 = 32 KB
     static constexpr uint32_t BAR_OFF = DS_OFF + 32768;
-    static constexpr int NUM_BARS = 20;
+    static constexpr int NUM_BARS = 10 + 5 * QS;
     static constexpr uint32_t MISC_OFF = BAR_OFF + 8 * NUM_BARS;
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
     // TMEM columns: S^T / P^T, dP^T, the dV and dK accumulators, the dQ partial
@@ -116,26 +120,43 @@ __device__ __forceinline__ uint32_t bwd_p_col(int kk) {
     return static_cast<uint32_t>((kk >> 2) * 64 + (kk & 3) * 8);
 }
 
-/* D_i = dO_i . O_i, lse2_i = LSE_i log2(e) (zero past N).  One warp per padded row. */
+/* D_i = dO_i . O_i, lse2_i = LSE_i log2(e) (zero past N).  D / 8 threads per
+ * padded row, each with one 16-byte load of O_i and of dO_i (every pointer is
+ * 16-byte aligned, checked on the host), so a warp reads whole rows; the
+ * partial sums of a row meet through shuffles among its lanes. */
+constexpr int BWD_PRE_THREADS = 256;
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(BWD_PRE_THREADS)
 bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                const float* __restrict__ lse, float* __restrict__ Dp, float* __restrict__ lse2,
                int N, int Np, int BH) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t prow = static_cast<int64_t>(blockIdx.x) * 8 + warp;     // over BH * Np
-    if (prow >= static_cast<int64_t>(BH) * Np) return;
-    const int bh = static_cast<int>(prow / Np), i = static_cast<int>(prow % Np);
+    constexpr int TPR = D / 8;                       // threads per row
+    constexpr int ROWS = BWD_PRE_THREADS / TPR;      // rows per block
+    const int part = threadIdx.x % TPR;
+    const int64_t prow = static_cast<int64_t>(blockIdx.x) * ROWS + threadIdx.x / TPR;  // over BH * Np
+    const bool valid = prow < static_cast<int64_t>(BH) * Np;   // the same for a row's lanes
+    int bh = 0, i = 0;
     float dsum = 0.0f;
-    if (i < N) {
-        const int64_t base = (static_cast<int64_t>(bh) * N + i) * D;
+    if (valid) {
+        bh = static_cast<int>(prow / Np);
+        i = static_cast<int>(prow % Np);
+        if (i < N) {
+            const int64_t off = (static_cast<int64_t>(bh) * N + i) * D + part * 8;
+            const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + off));
+            const uint4 g = __ldg(reinterpret_cast<const uint4*>(dout + off));
+            const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, gw[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
-        for (int c = lane; c < D; c += 32)
-            dsum += __bfloat162float(o[base + c]) * __bfloat162float(dout[base + c]);
+            for (int e = 0; e < 4; ++e) {
+                const float2 af = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&aw[e]));
+                const float2 gf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[e]));
+                dsum += af.x * gf.x;
+                dsum += af.y * gf.y;
+            }
+        }
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
-    if (lane == 0) {
+    for (int off = TPR / 2; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
+    if (valid && part == 0) {
         Dp[prow] = i < N ? dsum : 0.0f;
         lse2[prow] = i < N ? lse[static_cast<int64_t>(bh) * N + i] * LOG2E : 0.0f;
     }
@@ -215,18 +236,20 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t sK = base + C::K_OFF, sV = base + C::V_OFF, sDS = base + C::DS_OFF;
     const uint32_t bars = base + C::BAR_OFF;
     const uint32_t bar_kv = bars;
-    // Q_i and dO_i of a stage land, and are handed back, separately: the readout
-    // stages the first half of the dQ partial over Q_i and reduce-adds it first,
-    // so the next Q block can load while the second half (over dO_i) is staged
-    auto bar_full_q = [&](int s) { return bars + 8 + 8u * s; };
-    auto bar_empty = [&](int s) { return bars + 24 + 8u * s; };
-    const uint32_t bar_s = bars + 40, bar_p = bars + 48, bar_pt = bars + 56, bar_dqf = bars + 64;
-    const uint32_t bar_dkv = bars + 72, bar_drain = bars + 80, bar_dp = bars + 88;
-    auto bar_free_q = [&](int s) { return bars + 96 + 8u * s; };    // Q half of stage s handed back
-    const uint32_t bar_rd_q = bars + 112;                           // first half of the dQ tile staged
-    auto bar_full_do = [&](int s) { return bars + 120 + 8u * s; };
-    auto bar_free_do = [&](int s) { return bars + 136 + 8u * s; };  // dO half of stage s handed back
-    const uint32_t bar_rd_do = bars + 152;                          // second half staged
+    const uint32_t bar_s = bars + 8, bar_p = bars + 16, bar_pt = bars + 24, bar_dqf = bars + 32;
+    const uint32_t bar_dkv = bars + 40, bar_drain = bars + 48, bar_dp = bars + 56;
+    const uint32_t bar_rd_q = bars + 64;                            // first half of the dQ tile staged
+    const uint32_t bar_rd_do = bars + 72;                           // second half staged
+    // Per ring stage.  Q_i and dO_i of a stage land, and are handed back,
+    // separately: the readout stages the first half of the dQ partial over Q_i
+    // and reduce-adds it first, so the next Q block can load while the second
+    // half (over dO_i) is staged.
+    constexpr int QS = C::QS;
+    auto bar_full_q = [&](int s) { return bars + 80 + 8u * s; };
+    auto bar_full_do = [&](int s) { return bars + 80 + 8u * (QS + s); };
+    auto bar_empty = [&](int s) { return bars + 80 + 8u * (2 * QS + s); };    // dK_i has read Q_i
+    auto bar_free_q = [&](int s) { return bars + 80 + 8u * (3 * QS + s); };   // Q half handed back
+    auto bar_free_do = [&](int s) { return bars + 80 + 8u * (4 * QS + s); };  // dO half handed back
     uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::MISC_OFF);
     volatile uint32_t* const abort_flag = reinterpret_cast<volatile uint32_t*>(base_ptr + C::MISC_OFF + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -249,7 +272,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     if (threadIdx.x == 0) {
         mbar_init(bar_kv, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < QS; ++s) {
             mbar_init(bar_full_q(s), 1);
             mbar_init(bar_full_do(s), 1);
             mbar_init(bar_empty(s), 1);
@@ -290,15 +313,16 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             int issued_q = 0, issued_do = 0;
             for (int it = 0; it < nq; ++it) {
-                const int s = it & 1;
+                const int s = it % QS;
+                const uint32_t use = static_cast<uint32_t>(it / QS);
                 const int ib = ib0 + it;
-                if (!mbar_wait_inl(bar_free_q(s), ((it >> 1) & 1) ^ 1, abort_flag, wlim)) break;
+                if (!mbar_wait_inl(bar_free_q(s), (use & 1u) ^ 1u, abort_flag, wlim)) break;
                 mbar_arrive_expect_tx(bar_full_q(s), TILE);
                 for (int c = 0; c < C::CHUNKS; ++c)
                     tma_load_3d(&tm_q, base + C::Q_OFF + s * TILE + c * CHUNK_BYTES, bar_full_q(s),
                                 c * CHUNK_ELEMS, ib * BLOCK_M, bh);
                 ++issued_q;
-                if (!mbar_wait_inl(bar_free_do(s), ((it >> 1) & 1) ^ 1, abort_flag, wlim)) break;
+                if (!mbar_wait_inl(bar_free_do(s), (use & 1u) ^ 1u, abort_flag, wlim)) break;
                 mbar_arrive_expect_tx(bar_full_do(s), TILE);
                 for (int c = 0; c < C::CHUNKS; ++c)
                     tma_load_3d(&tm_do, base + C::DO_OFF + s * TILE + c * CHUNK_BYTES, bar_full_do(s),
@@ -307,13 +331,13 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             // every copy this thread issued lands before the CTA can exit
             mbar_drain_wait_inl(bar_kv, 0, wlim);
-            for (int b = 1; b <= (issued_q < 2 ? issued_q : 2); ++b) {
+            for (int b = 1; b <= (issued_q < QS ? issued_q : QS); ++b) {
                 const int it = issued_q - b;
-                mbar_drain_wait_inl(bar_full_q(it & 1), (it >> 1) & 1, wlim);
+                mbar_drain_wait_inl(bar_full_q(it % QS), (it / QS) & 1, wlim);
             }
-            for (int b = 1; b <= (issued_do < 2 ? issued_do : 2); ++b) {
+            for (int b = 1; b <= (issued_do < QS ? issued_do : QS); ++b) {
                 const int it = issued_do - b;
-                mbar_drain_wait_inl(bar_full_do(it & 1), (it >> 1) & 1, wlim);
+                mbar_drain_wait_inl(bar_full_do(it % QS), (it / QS) & 1, wlim);
             }
         }
         __syncwarp();
@@ -339,7 +363,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mma_commit(bar_s);
             }
             for (int it = 0; it < nq && ok; ++it) {
-                const int s = it & 1;
+                const int s = it % QS;
                 const uint32_t sq = base + C::Q_OFF + s * TILE, sdo = base + C::DO_OFF + s * TILE;
                 if (C::DQ_OVER_DP && it > 0) {
                     // dP^T overwrites the previous dQ partial: wait until it was read out
@@ -347,7 +371,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (!ok) break;
                     tc_fence_after();
                 }
-                ok = mbar_wait_inl(bar_full_do(s), (it >> 1) & 1, abort_flag, wlim);   // dO_i landed
+                ok = mbar_wait_inl(bar_full_do(s), (it / QS) & 1, abort_flag, wlim);   // dO_i landed
                 if (!ok) break;
                 issue_qk<D>(tb, vd, sdesc_sw128(sdo, 16, 1024), ID_KQ);         // dP^T = V dO^T
                 mma_commit(bar_dp);
@@ -356,8 +380,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 // the next S^T over P^T: the tensor core reads P^T for dV first
                 auto issue_next_s = [&]() -> bool {
                     if (it + 1 >= nq) return true;
-                    const int s1 = s ^ 1;
-                    if (!mbar_wait_inl(bar_full_q(s1), ((it + 1) >> 1) & 1, abort_flag, wlim)) return false;
+                    const int s1 = (it + 1) % QS;
+                    if (!mbar_wait_inl(bar_full_q(s1), ((it + 1) / QS) & 1, abort_flag, wlim)) return false;
                     tc_fence_after();
                     issue_qk<D>(ta, kd, sdesc_sw128(base + C::Q_OFF + s1 * TILE, 16, 1024), ID_KQ);
                     mma_commit(bar_s);
@@ -420,8 +444,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
         const bool leader = threadIdx.x == BWD_READ_WARP0 * 32;
         for (int it = 0; it < nq; ++it) {
-            const int s = it & 1, ib = ib0 + it;
-            bool ok = mbar_wait_inl(bar_empty(s), (it >> 1) & 1, abort_flag, wlim);   // dK_i done
+            const int s = it % QS, ib = ib0 + it;
+            bool ok = mbar_wait_inl(bar_empty(s), (it / QS) & 1, abort_flag, wlim);   // dK_i done
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();

@@ -1695,7 +1695,9 @@ int bwd_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
     const int64_t prows = static_cast<int64_t>(prm.BH) * prm.Np;
     if (cudaMemsetAsync(prm.dq_acc, 0, static_cast<size_t>(prows) * D * 4, stream) != cudaSuccess)
         return ATTN_ERR_CUDA;
-    bwd_pre_kernel<D><<<static_cast<unsigned>((prows + 7) / 8), 256, 0, stream>>>(
+    constexpr int pre_rows = BWD_PRE_THREADS / (D / 8);
+    bwd_pre_kernel<D><<<static_cast<unsigned>((prows + pre_rows - 1) / pre_rows), BWD_PRE_THREADS, 0,
+                        stream>>>(
         o, dout, lse, const_cast<float*>(prm.Dp), const_cast<float*>(prm.lse2), prm.N, prm.Np,
         prm.BH);
     kern<<<static_cast<unsigned>(prm.nblk * prm.BH), BWD_THREADS, SMEM, stream>>>(mq, mk, mv, mdo, prm);

@@ -520,6 +520,12 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int64_t row0 = static_cast<int64_t>(bh) * p.Np + ib * BLOCK_M + 64 * h;
             const float* lse2 = p.lse2 + row0;
             const float* dvec = p.Dp + row0;
+            if (lane < 4 && it + 1 < nq) {
+                // the next Q block's LSE and D values (two 128-byte lines each) into L1
+                // now, so that their first reads next step do not wait on L2
+                const float* nx = (lane < 2 ? lse2 : dvec) + BLOCK_M + 32 * (lane & 1);
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(nx));
+            }
             // on the diagonal block key r is masked for the queries before it:
             // column ch * 32 + e of this half is masked when it is < mask_lim
             const bool diag = CAUSAL && ib == jb;

@@ -478,13 +478,15 @@ __device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& p0, fl
 }
 
 /* Which column pairs of a score row take the polynomial (bit k%8 of the mask
- * for pair k); the rest use the MUFU ex2.  Measured per head dimension: at
- * d = 64 (half the tensor work per exponential of d = 128) 2 of 8 pairs on the
- * FMA pipe was fastest; at d = 128 and for e4m3 every fraction tried was
- * slower than none. */
+ * for pair k); the rest use the MUFU ex2.  2 of 8 pairs on the FMA pipe where
+ * the exponentials outweigh the tensor work per block: bf16 at d = 64 (+2.3 %)
+ * and e4m3 at both head dimensions (+8.7 % on causal N = 8192 d = 128, +5.8 %
+ * on N = 2048 d = 64; 1/8 gains half of that, 4/8 and 5/8 lose).  For bf16 at
+ * d = 128, where MUFU and tensor work per block are equal, every fraction
+ * measured was slower than or equal to none. */
 template <int D, bool FP8>
 __device__ __forceinline__ constexpr uint32_t exp2_poly_mask() {
-    return (D == 64 && !FP8) ? 0x11u : 0x00u;
+    return (D == 64 || FP8) ? 0x11u : 0x00u;
 }
 
 /* Two fp32 -> one bf16x2 word, round to nearest even; `lo` in bits 0-15. */

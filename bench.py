@@ -397,6 +397,24 @@ def run_cuda(args, w):
                   "kernel_median_us": 1e3 * statistics.median(kernel_ms),
                   "calls": args.latency_calls,
                   "what": "host wall time of attn_fwd + stream synchronize, one call at a time"}
+        # the same call captured once in a CUDA graph and replayed: the host work of
+        # a call (checks, tensor maps, launch) is paid at capture only
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            shard.attn_fwd_heads(qd, kd, vd, causal=w.causal, scale=w.scale, out=o, lse=lse)
+        cap = torch.cuda.current_stream()
+        for _ in range(3):
+            graph.replay()
+        cap.synchronize()
+        replay = []
+        for _ in range(args.latency_calls):
+            t0 = time.perf_counter()
+            graph.replay()
+            cap.synchronize()
+            replay.append((time.perf_counter() - t0) * 1e6)
+        lat_us["graph_replay_median_us"] = statistics.median(replay)
+        lat_us["graph_what"] = "host wall time of CUDAGraph.replay() + synchronize of one captured attn_fwd"
+        del graph
 
     # ---- optional gather of every rank's O and LSE onto all ranks (NCCL all-gather)
     gather = None

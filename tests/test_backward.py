@@ -117,6 +117,32 @@ def test_backward_headline_workload_two_heads():
 
 
 @pytest.mark.gpu
+def test_backward_d64_workload_two_heads():
+    """The d = 64 configuration bench.py --pass bwd times (B=8, H=16, N=2048,
+    non-causal): 16 Q blocks per K/V block, so every stage of the d = 64 ring
+    (four stages) is reused four times; checked in full on the first and the
+    last head."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    w = inputs.WORKLOADS["b8h16_n2048_d64"]
+    q, k, v = inputs.workload_inputs(w)
+    dout = inputs.make_qkv(w.B, w.H, w.N, w.d, w.seed + 100)[0]
+    _check(q, k, v, dout, w.causal, w.scale, w.name, heads=[0, w.B * w.H - 1])
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_large_logits_d64(causal):
+    """Peaked softmax at d = 64, over more Q blocks (N = 1100, ragged tail) than
+    the ring has stages."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    q, k, v = inputs.make_qkv(1, 2, 1100, 64, seed=49, qk_std=4.0, v_dist="uniform")
+    dout = inputs.make_qkv(1, 2, 1100, 64, seed=50)[0]
+    _check(q, k, v, dout, causal, 1 / math.sqrt(64), f"large logits d64 causal={causal}")
+
+
+@pytest.mark.gpu
 def test_backward_deterministic_dk_dv():
     """dK and dV are written once per K/V block (no atomics): bit-identical reruns."""
     if not torch.cuda.is_available():

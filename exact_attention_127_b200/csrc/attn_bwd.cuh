@@ -17,25 +17,28 @@
  * bwd_main_kernel  one CTA per (head, 128-row K/V block j), looping over the Q
  *                  blocks i that see block j; CTAs start longest first within
  *                  groups of heads.  K_j and V_j stay in shared memory;
- *                  Q_i and dO_i stream through a 2-stage TMA ring.  Per i, on
- *                  the tensor cores (TMEM accumulators):
+ *                  Q_i and dO_i stream through a TMA ring (2 stages at d = 128,
+ *                  4 at d = 64).  Per i, on the tensor cores (TMEM accumulators):
  *                      S^T  = K_j Q_i^T   -> TMEM A      dP^T = V_j dO_i^T -> TMEM B
  *                  warps 0-7 (thread = K/V row = TMEM lane; warps w and w+4 share
  *                  the lanes and split the 128 queries in halves) turn S^T into
  *                  P^T (bf16, packed over the first half of its own columns of
- *                  TMEM A) and, once dP^T is there, scale * dS (bf16) into shared
- *                  memory; then
- *                      dQ_i partial = dS K_j          (A, B from shared memory) -> TMEM dQ
+ *                  TMEM A); then, while they form scale * dS (bf16) into shared
+ *                  memory once dP^T is there,
  *                      dV_j += P^T dO_i               (A from TMEM)
  *                      S^T of block i+1               (overwrites P^T: MMAs run in issue order)
+ *                  and once dS is stored
+ *                      dQ_i partial = dS K_j          (A, B from shared memory) -> TMEM dQ
  *                      dK_j += dS^T Q_i               (A, B from shared memory)
- *                  (at d = 64, where dQ has TMEM columns of its own, dV_i and the
- *                  next S^T go as soon as P^T is in TMEM, while warps 0-7 form
- *                  dS, and dQ_i, dK_j follow)
- *                  Warps 12-15 (thread = query row) copy the dQ partial into the
- *                  freed Q_i / dO_i stage, and one of them adds it into the fp32
- *                  accumulator with TMA bulk reduce-adds, while warps 0-7 already
- *                  work on block i+1.  At the end warps 0-7 write dK_j, dV_j.
+ *                  At d = 128 the dQ partial lies over dP^T, whose columns the next
+ *                  block's dP^T needs: warps 12-15 (thread = query row) take it out
+ *                  of TMEM as soon as it lands, staging a quarter over dO_i (which
+ *                  dV_i and dP^T_i have read) and holding the rest in registers,
+ *                  release the columns, and stage the rest over Q_i once dK_i has
+ *                  read it.  At d = 64 (own columns) they stage it over the freed
+ *                  Q_i / dO_i stage.  One of them adds the staged halves into the
+ *                  fp32 accumulator with TMA bulk reduce-adds, while warps 0-7
+ *                  already work on block i+1.  At the end warps 0-7 write dK_j, dV_j.
  *                  Warp 8 issues the TMA loads, warp 9 the MMAs; setmaxnreg
  *                  gives the P/dS warps the registers of the others.
  * bwd_post_kernel  dQ accumulator -> bf16.
@@ -53,12 +56,14 @@ constexpr int BWD_MMA_WARP = 9;
 constexpr int BWD_READ_WARP0 = 12;
 constexpr int BWD_READERS = 128;
 /* Register split (setmaxnreg) of the 512 x 128 registers the launch holds:
- * the P/dS warpgroups rise to 176, the TMA/MMA warpgroup (with the two warps
- * that have no role) drops to 56 and the readout warpgroup to 104. */
+ * the P/dS warpgroups rise to 168, the TMA/MMA warpgroup (with the two warps
+ * that have no role) drops to 56 and the readout warpgroup to 120 (96 columns
+ * of the dQ partial held at once: with 512 threads ptxas allows no instruction
+ * more than 128 live registers). */
 constexpr int BWD_LAUNCH_REGS = 128;  // per thread at launch (checked on the host before launching)
-constexpr int BWD_COMPUTE_REGS = 176;
+constexpr int BWD_COMPUTE_REGS = 168;
 constexpr int BWD_CTRL_REGS = 56;
-constexpr int BWD_READ_REGS = 104;
+constexpr int BWD_READ_REGS = 120;
 static_assert(2 * 128 * BWD_COMPUTE_REGS + 128 * BWD_CTRL_REGS + 128 * BWD_READ_REGS ==
                   BWD_THREADS * BWD_LAUNCH_REGS,
               "register split");
@@ -89,7 +94,7 @@ struct BwdCfg {
     static constexpr uint32_t DO_OFF = Q_OFF + QS * TILE;       // [QS] stages
     static constexpr uint32_t DS_OFF = DO_OFF + QS * TILE;      // 128 x 128 bf16 = 32 KB
     static constexpr uint32_t BAR_OFF = DS_OFF + 32768;
-    static constexpr int NUM_BARS = 10 + 5 * QS;
+    static constexpr int NUM_BARS = 11 + 5 * QS;
     static constexpr uint32_t MISC_OFF = BAR_OFF + 8 * NUM_BARS;
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
     // TMEM columns: S^T / P^T, dP^T, the dV and dK accumulators, the dQ partial
@@ -97,14 +102,6 @@ struct BwdCfg {
     static constexpr uint32_t RA = 0, RB = 128, DV_COL = 256, DK_COL = 256 + D;
     static constexpr uint32_t DQ_COL = (256 + 2 * D + D <= 512) ? 256 + 2 * D : RB;
     static constexpr bool DQ_OVER_DP = DQ_COL == RB;
-    // dV_i and the next S^T as soon as P^T is in TMEM, before dS: faster where
-    // dQ has columns of its own (D = 64); at D = 128 the later order measured faster
-    static constexpr bool EARLY_NEXT_S = !DQ_OVER_DP;
-    // The Q half of a ring stage goes back to the producer as soon as its dQ
-    // reduce has read it (D = 64), or only once the dO half is staged too
-    // (D = 128, where the dQ columns lie under dP^T: stalling the readout warp on
-    // the first reduce would delay their release and with it the next dP^T)
-    static constexpr bool EAGER_Q_FREE = !DQ_OVER_DP;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
@@ -240,16 +237,17 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t bar_dkv = bars + 40, bar_drain = bars + 48, bar_dp = bars + 56;
     const uint32_t bar_rd_q = bars + 64;                            // first half of the dQ tile staged
     const uint32_t bar_rd_do = bars + 72;                           // second half staged
+    const uint32_t bar_dq = bars + 80;                              // the dQ partial is in TMEM
     // Per ring stage.  Q_i and dO_i of a stage land, and are handed back,
     // separately: the readout stages the first half of the dQ partial over Q_i
     // and reduce-adds it first, so the next Q block can load while the second
     // half (over dO_i) is staged.
     constexpr int QS = C::QS;
-    auto bar_full_q = [&](int s) { return bars + 80 + 8u * s; };
-    auto bar_full_do = [&](int s) { return bars + 80 + 8u * (QS + s); };
-    auto bar_empty = [&](int s) { return bars + 80 + 8u * (2 * QS + s); };    // dK_i has read Q_i
-    auto bar_free_q = [&](int s) { return bars + 80 + 8u * (3 * QS + s); };   // Q half handed back
-    auto bar_free_do = [&](int s) { return bars + 80 + 8u * (4 * QS + s); };  // dO half handed back
+    auto bar_full_q = [&](int s) { return bars + 88 + 8u * s; };
+    auto bar_full_do = [&](int s) { return bars + 88 + 8u * (QS + s); };
+    auto bar_empty = [&](int s) { return bars + 88 + 8u * (2 * QS + s); };    // dK_i has read Q_i
+    auto bar_free_q = [&](int s) { return bars + 88 + 8u * (3 * QS + s); };   // Q half handed back
+    auto bar_free_do = [&](int s) { return bars + 88 + 8u * (4 * QS + s); };  // dO half handed back
     uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::MISC_OFF);
     volatile uint32_t* const abort_flag = reinterpret_cast<volatile uint32_t*>(base_ptr + C::MISC_OFF + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -283,6 +281,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(bar_rd_do, BWD_READERS);
         mbar_init(bar_s, 1);
         mbar_init(bar_dp, 1);
+        mbar_init(bar_dq, 1);
         mbar_init(bar_p, BWD_COMPUTE);
         mbar_init(bar_pt, BWD_COMPUTE);
         mbar_init(bar_dqf, BWD_READERS);
@@ -387,33 +386,25 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mma_commit(bar_s);
                     return true;
                 };
-                if constexpr (C::EARLY_NEXT_S) {
-                    // D = 64: dV and the next S^T while warps 0-7 still form dS
-                    ok = mbar_wait_inl(bar_pt, it & 1, abort_flag, wlim);        // P^T in TMEM
+                // dV_i and the next S^T as soon as P^T is in TMEM, while warps 0-7
+                // still form dS; then dQ_i and dK_i once dS is in shared memory
+                ok = mbar_wait_inl(bar_pt, it & 1, abort_flag, wlim);        // P^T in TMEM
+                if (!ok) break;
+                tc_fence_after();
+                bwd_issue_dv(tdv, ta, do_mn, ID_ACC, it > 0);
+                ok = issue_next_s();
+                if (!ok) break;
+                ok = mbar_wait_inl(bar_p, it & 1, abort_flag, wlim);         // dS in shared memory
+                if (!ok) break;
+                tc_fence_after();
+                if (!C::DQ_OVER_DP && it > 0) {
+                    // the previous dQ partial has its own columns: read out yet?
+                    ok = mbar_wait_inl(bar_dqf, (it - 1) & 1, abort_flag, wlim);
                     if (!ok) break;
                     tc_fence_after();
-                    bwd_issue_dv(tdv, ta, do_mn, ID_ACC, it > 0);
-                    ok = issue_next_s();
-                    if (!ok) break;
-                    ok = mbar_wait_inl(bar_p, it & 1, abort_flag, wlim);         // dS in shared memory
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (it > 0) {
-                        ok = mbar_wait_inl(bar_dqf, (it - 1) & 1, abort_flag, wlim);
-                        if (!ok) break;
-                        tc_fence_after();
-                    }
-                    bwd_issue_dq(tdq, ds_mn, k_mn, ID_DQ);
-                } else {
-                    // D = 128: dQ (over dP^T) first, then dV and the next S^T
-                    ok = mbar_wait_inl(bar_p, it & 1, abort_flag, wlim);
-                    if (!ok) break;
-                    tc_fence_after();
-                    bwd_issue_dq(tdq, ds_mn, k_mn, ID_DQ);
-                    bwd_issue_dv(tdv, ta, do_mn, ID_ACC, it > 0);
-                    ok = issue_next_s();
-                    if (!ok) break;
                 }
+                bwd_issue_dq(tdq, ds_mn, k_mn, ID_DQ);
+                if constexpr (C::DQ_OVER_DP) mma_commit(bar_dq);   // the readout may take it now
 #pragma unroll 1
                 for (int kk = 0; kk < BLOCK_M / 16; ++kk) {
                     const uint64_t off_mn = static_cast<uint64_t>((kk * 16 * 128) >> 4);
@@ -431,28 +422,91 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     } else if (warp >= BWD_READ_WARP0) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(BWD_READ_REGS) : "memory");
         /* ---------------- warps 12-15: the dQ partial of Q block i ----------------
-         * Once dK_i has read Q_i (so the stage of Q_i and dO_i is free), thread
-         * r = query row copies its row of the partial from TMEM into that stage,
-         * laid out as the accumulator tile (first half over Q_i, second over
-         * dO_i), and releases the dQ columns.  One thread adds each half into the
-         * fp32 accumulator with a TMA bulk reduce-add as soon as it is staged, and
-         * hands that half of the stage back to the producer once the reduce has
-         * read it, so the next Q block's load need not wait for the dO half: no
-         * atomics through the SM's load/store path. */
+         * Thread r = query row copies its row of the partial from TMEM into the
+         * Q_i / dO_i stage, laid out as the accumulator tile, and releases the dQ
+         * columns; at D = 128 early, as described below.  One thread adds each half
+         * into the fp32 accumulator with a TMA bulk reduce-add as soon as it is
+         * staged, and hands that half of the stage back to the producer once the
+         * reduce has read it: no atomics through the SM's load/store path. */
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
         const bool leader = threadIdx.x == BWD_READ_WARP0 * 32;
         for (int it = 0; it < nq; ++it) {
             const int s = it % QS, ib = ib0 + it;
+            if constexpr (C::DQ_OVER_DP) {
+                /* dQ_i has landed over dP^T_i.  dV_i and dP^T_i, issued before it, have
+                 * read dO_i, so the first half of the partial goes over dO_i at once and
+                 * is reduce-added; the second half is then held in registers, the dQ
+                 * columns (the next dP^T) are released, and it goes over Q_i once dK_i
+                 * has read Q_i. */
+                bool ok = mbar_wait_inl(bar_dq, it & 1, abort_flag, wlim);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t sq = base + C::Q_OFF + s * TILE, sdo = base + C::DO_OFF + s * TILE;
+                float* tile = p.dq_acc + (static_cast<int64_t>(bh) * p.nblk + ib) * (BLOCK_M * D);
+                // chunk 0 goes over dO_i first; chunks 1-3 (96 columns, as many as a thread
+                // of this warpgroup holds) are then read and the columns released
+                {
+                    uint32_t v[32];
+                    tmem_ld32_wait(lane_base + C::DQ_COL, v);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const uint32_t dst = sdo + (e * BLOCK_M + r) * 16;
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[4 * e]),
+                                     "r"(v[4 * e + 1]), "r"(v[4 * e + 2]), "r"(v[4 * e + 3]) : "memory");
+                    }
+                }
+                uint32_t hv[96];
+#pragma unroll
+                for (int ch = 0; ch < 3; ++ch)
+                    tmem_ld32_wait(lane_base + C::DQ_COL + 32 + ch * 32, hv + 32 * ch);
+                tc_fence_before();
+                mbar_arrive(bar_dqf);                 // every column read
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {         // chunk 1: the rest of the dO_i half
+                    const uint32_t dst = sdo + ((8 + e) * BLOCK_M + r) * 16;
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(hv[4 * e]),
+                                 "r"(hv[4 * e + 1]), "r"(hv[4 * e + 2]), "r"(hv[4 * e + 3]) : "memory");
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_arrive(bar_rd_do);
+                if (leader) {
+                    if (!mbar_wait_inl(bar_rd_do, it & 1, abort_flag, wlim)) break;
+                    bulk_reduce_add_f32(tile, sdo, TILE);
+                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                }
+                ok = mbar_wait_inl(bar_empty(s), (it / QS) & 1, abort_flag, wlim);   // dK_i done
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+#pragma unroll
+                for (int g = 0; g < D / 8; ++g) {
+                    const uint32_t dst = sq + (g * BLOCK_M + r) * 16;
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(hv[32 + 4 * g]),
+                                 "r"(hv[32 + 4 * g + 1]), "r"(hv[32 + 4 * g + 2]), "r"(hv[32 + 4 * g + 3]) : "memory");
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_arrive(bar_rd_q);
+                if (leader) {
+                    if (!mbar_wait_inl(bar_rd_q, it & 1, abort_flag, wlim)) break;
+                    bulk_reduce_add_f32(tile + TILE / 4, sq, TILE);
+                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");   // dO half read
+                    mbar_arrive(bar_free_do(s));
+                    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // Q half read
+                    mbar_arrive(bar_free_q(s));
+                }
+                continue;
+            }
+            // D = 64: once dK_i has read Q_i, half 0 (column groups [0, D/8)) over Q_i,
+            // half 1 over dO_i, each reduce-added as soon as it is staged
             bool ok = mbar_wait_inl(bar_empty(s), (it / QS) & 1, abort_flag, wlim);   // dK_i done
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
             const uint32_t sq = base + C::Q_OFF + s * TILE, sdo = base + C::DO_OFF + s * TILE;
             float* tile = p.dq_acc + (static_cast<int64_t>(bh) * p.nblk + ib) * (BLOCK_M * D);
-            // half 0 (column groups [0, D/8)) over Q_i, half 1 over dO_i; each half is
-            // reduce-added, and its stage half handed back, as soon as it is staged
 #pragma unroll 1
             for (int half = 0; half < 2 && ok; ++half) {
                 const uint32_t dst0 = half ? sdo : sq;
@@ -479,19 +533,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (!mbar_wait_inl(bar_rd, it & 1, abort_flag, wlim)) { ok = false; break; }
                     bulk_reduce_add_f32(tile + half * (TILE / 4), dst0, TILE);
                     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-                    if (half == 0) {
-                        if constexpr (C::EAGER_Q_FREE) {
-                            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // Q half read
-                            mbar_arrive(bar_free_q(s));
-                        }
-                    } else {
-                        if constexpr (!C::EAGER_Q_FREE) {
-                            asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");   // Q half read
-                            mbar_arrive(bar_free_q(s));
-                        }
-                        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // dO half read
-                        mbar_arrive(bar_free_do(s));
-                    }
+                    // each half of the stage goes back as soon as its reduce has read it
+                    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                    mbar_arrive(half ? bar_free_do(s) : bar_free_q(s));
                 }
             }
             if (!ok) break;
@@ -557,11 +601,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 tmem_st16(lane_base + C::RA + 64 * h + 16 * ch, pk);
             }
-            if constexpr (C::EARLY_NEXT_S) {
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar_pt);    // P^T is in TMEM: dV and the next S^T may go
-            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar_pt);    // P^T is in TMEM: dV and the next S^T may go
             ok = mbar_wait_inl(bar_dp, it & 1, abort_flag, wlim);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
@@ -601,7 +643,6 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                  "r"(dk[4 * u + 3]) : "memory");
                 }
             }
-            if constexpr (!C::EARLY_NEXT_S) tmem_wait_st();   // the P^T stores
             tc_fence_before();
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // dS visible to the MMA
             mbar_arrive(bar_p);

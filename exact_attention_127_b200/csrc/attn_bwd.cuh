@@ -34,9 +34,11 @@
  *                  block's dP^T needs: warps 12-15 (thread = query row) take it out
  *                  of TMEM as soon as it lands, staging a quarter over dO_i (which
  *                  dV_i and dP^T_i have read) and holding the rest in registers,
- *                  release the columns, and stage the rest over Q_i once dK_i has
- *                  read it.  At d = 64 (own columns) they stage it over the freed
- *                  Q_i / dO_i stage.  One of them adds the staged halves into the
+ *                  and release the columns; the second half of the partial follows
+ *                  the first through the dO_i half, so the Q_i half of the stage
+ *                  goes back as soon as dK_i has read it and the next Q block's
+ *                  load waits for no reduce.  At d = 64 (own columns) they stage
+ *                  it over the freed Q_i / dO_i stage.  One of them adds the staged halves into the
  *                  fp32 accumulator with TMA bulk reduce-adds, while warps 0-7
  *                  already work on block i+1.  At the end warps 0-7 write dK_j, dV_j.
  *                  Warp 8 issues the TMA loads, warp 9 the MMAs; setmaxnreg
@@ -94,7 +96,7 @@ struct BwdCfg {
     static constexpr uint32_t DO_OFF = Q_OFF + QS * TILE;       // [QS] stages
     static constexpr uint32_t DS_OFF = DO_OFF + QS * TILE;      // 128 x 128 bf16 = 32 KB
     static constexpr uint32_t BAR_OFF = DS_OFF + 32768;
-    static constexpr int NUM_BARS = 11 + 5 * QS;
+    static constexpr int NUM_BARS = 12 + 5 * QS;
     static constexpr uint32_t MISC_OFF = BAR_OFF + 8 * NUM_BARS;
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
     // TMEM columns: S^T / P^T, dP^T, the dV and dK accumulators, the dQ partial
@@ -238,16 +240,17 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t bar_rd_q = bars + 64;                            // first half of the dQ tile staged
     const uint32_t bar_rd_do = bars + 72;                           // second half staged
     const uint32_t bar_dq = bars + 80;                              // the dQ partial is in TMEM
+    const uint32_t bar_sdo = bars + 88;                             // dO half read by the first reduce
     // Per ring stage.  Q_i and dO_i of a stage land, and are handed back,
     // separately: the readout stages the first half of the dQ partial over Q_i
     // and reduce-adds it first, so the next Q block can load while the second
     // half (over dO_i) is staged.
     constexpr int QS = C::QS;
-    auto bar_full_q = [&](int s) { return bars + 88 + 8u * s; };
-    auto bar_full_do = [&](int s) { return bars + 88 + 8u * (QS + s); };
-    auto bar_empty = [&](int s) { return bars + 88 + 8u * (2 * QS + s); };    // dK_i has read Q_i
-    auto bar_free_q = [&](int s) { return bars + 88 + 8u * (3 * QS + s); };   // Q half handed back
-    auto bar_free_do = [&](int s) { return bars + 88 + 8u * (4 * QS + s); };  // dO half handed back
+    auto bar_full_q = [&](int s) { return bars + 96 + 8u * s; };
+    auto bar_full_do = [&](int s) { return bars + 96 + 8u * (QS + s); };
+    auto bar_empty = [&](int s) { return bars + 96 + 8u * (2 * QS + s); };    // dK_i has read Q_i
+    auto bar_free_q = [&](int s) { return bars + 96 + 8u * (3 * QS + s); };   // Q half handed back
+    auto bar_free_do = [&](int s) { return bars + 96 + 8u * (4 * QS + s); };  // dO half handed back
     uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::MISC_OFF);
     volatile uint32_t* const abort_flag = reinterpret_cast<volatile uint32_t*>(base_ptr + C::MISC_OFF + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -282,6 +285,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(bar_s, 1);
         mbar_init(bar_dp, 1);
         mbar_init(bar_dq, 1);
+        mbar_init(bar_sdo, 1);
         mbar_init(bar_p, BWD_COMPUTE);
         mbar_init(bar_pt, BWD_COMPUTE);
         mbar_init(bar_dqf, BWD_READERS);
@@ -437,9 +441,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if constexpr (C::DQ_OVER_DP) {
                 /* dQ_i has landed over dP^T_i.  dV_i and dP^T_i, issued before it, have
                  * read dO_i, so the first half of the partial goes over dO_i at once and
-                 * is reduce-added; the second half is then held in registers, the dQ
-                 * columns (the next dP^T) are released, and it goes over Q_i once dK_i
-                 * has read Q_i. */
+                 * is reduce-added; the second half is held in registers meanwhile, the
+                 * dQ columns (the next dP^T) are released, and it follows through the
+                 * dO_i half once the first reduce has read it. */
                 bool ok = mbar_wait_inl(bar_dq, it & 1, abort_flag, wlim);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
@@ -472,30 +476,35 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 mbar_arrive(bar_rd_do);
+                // the Q_i half of the stage is not staged into: it goes back once dK_i
+                // has read it; the second half of the partial follows the first through
+                // the dO_i half once the first reduce has read it
                 if (leader) {
-                    if (!mbar_wait_inl(bar_rd_do, it & 1, abort_flag, wlim)) break;
-                    bulk_reduce_add_f32(tile, sdo, TILE);
-                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                    if (mbar_wait_inl(bar_rd_do, it & 1, abort_flag, wlim)) {
+                        bulk_reduce_add_f32(tile, sdo, TILE);
+                        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                    }
+                    if (mbar_wait_inl(bar_empty(s), (it / QS) & 1, abort_flag, wlim))   // dK_i done
+                        mbar_arrive(bar_free_q(s));
+                    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // first half read
+                    mbar_arrive(bar_sdo);
                 }
-                ok = mbar_wait_inl(bar_empty(s), (it / QS) & 1, abort_flag, wlim);   // dK_i done
+                ok = mbar_wait_inl(bar_sdo, it & 1, abort_flag, wlim);            // dO_i half free again
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
 #pragma unroll
                 for (int g = 0; g < D / 8; ++g) {
-                    const uint32_t dst = sq + (g * BLOCK_M + r) * 16;
+                    const uint32_t dst = sdo + (g * BLOCK_M + r) * 16;
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(hv[32 + 4 * g]),
                                  "r"(hv[32 + 4 * g + 1]), "r"(hv[32 + 4 * g + 2]), "r"(hv[32 + 4 * g + 3]) : "memory");
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 mbar_arrive(bar_rd_q);
-                if (leader) {
-                    if (!mbar_wait_inl(bar_rd_q, it & 1, abort_flag, wlim)) break;
-                    bulk_reduce_add_f32(tile + TILE / 4, sq, TILE);
+                if (leader && mbar_wait_inl(bar_rd_q, it & 1, abort_flag, wlim)) {
+                    bulk_reduce_add_f32(tile + TILE / 4, sdo, TILE);
                     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-                    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");   // dO half read
+                    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // second half read
                     mbar_arrive(bar_free_do(s));
-                    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // Q half read
-                    mbar_arrive(bar_free_q(s));
                 }
                 continue;
             }

@@ -566,13 +566,21 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bool ok = true;
         for (int it = 0; it < nq; ++it) {
             const int ib = ib0 + it;
+            const int64_t row0 = static_cast<int64_t>(bh) * p.Np + ib * BLOCK_M + 64 * h;
+            const float* lse2 = p.lse2 + row0;
+            const float* dvec = p.Dp + row0;
+            // at D = 64 the LSE values of this half go out before the wait for S^T,
+            // which hides their latency (an L2 round trip under the dQ reduce-adds); at
+            // D = 128 the P/dS warps are not what the step waits for, and loading early
+            // measured slower there
+            constexpr int EARLY = D == 64 ? 16 : 0;
+            float4 l4e[16];
+#pragma unroll
+            for (int e = 0; e < EARLY; ++e) l4e[e] = __ldg(reinterpret_cast<const float4*>(lse2) + e);
             ok = mbar_wait_inl(bar_s, it & 1, abort_flag, wlim);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            const int64_t row0 = static_cast<int64_t>(bh) * p.Np + ib * BLOCK_M + 64 * h;
-            const float* lse2 = p.lse2 + row0;
-            const float* dvec = p.Dp + row0;
             if (lane < 4 && it + 1 < nq) {
                 // the next Q block's LSE and D values (two 128-byte lines each) into L1
                 // now, so that their first reads next step do not wait on L2
@@ -591,7 +599,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {
-                    const float4 l4 = __ldg(reinterpret_cast<const float4*>(lse2 + ch * 32 + e));
+                    const float4 l4 = EARLY ? l4e[ch * 8 + e / 4]
+                                            : __ldg(reinterpret_cast<const float4*>(lse2 + ch * 32 + e));
                     // c s - lse2 on pairs (f32x2: the same rounding as scalar fmaf)
                     float x[4];
                     f2unpack(ffma2(f2pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2,
@@ -613,6 +622,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar_pt);    // P^T is in TMEM: dV and the next S^T may go
+            float4 d4e[16];         // likewise the D values before the wait for dP^T
+#pragma unroll
+            for (int e = 0; e < EARLY; ++e) d4e[e] = __ldg(reinterpret_cast<const float4*>(dvec) + e);
             ok = mbar_wait_inl(bar_dp, it & 1, abort_flag, wlim);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
@@ -628,7 +640,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 uint32_t dk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {
-                    const float4 d4 = __ldg(reinterpret_cast<const float4*>(dvec + ch * 32 + e));
+                    const float4 d4 = EARLY ? d4e[ch * 8 + e / 4]
+                                            : __ldg(reinterpret_cast<const float4*>(dvec + ch * 32 + e));
                     // scale * P (dP - D) on pairs, in the scalar order (f32x2 rounds alike)
                     float dd[4];
                     const int j = ch * 32 + e;

@@ -131,6 +131,18 @@ def test_backward_d64_workload_two_heads():
 
 
 @pytest.mark.gpu
+def test_backward_d64_more_blocks_than_sms_all_heads():
+    """More K/V blocks than SMs at d = 64, non-causal: 40 heads of 9 K/V blocks
+    (N = 1100, ragged tail) make 360 CTAs, so each SM runs two or three of them in
+    turn, and every head is checked in full."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    q, k, v = inputs.make_qkv(2, 20, 1100, 64, seed=51)
+    dout = inputs.make_qkv(2, 20, 1100, 64, seed=52)[0]
+    _check(q, k, v, dout, False, 1 / math.sqrt(64), "d64, 360 K/V blocks, all heads")
+
+
+@pytest.mark.gpu
 @pytest.mark.parametrize("causal", [False, True])
 def test_backward_large_logits_d64(causal):
     """Peaked softmax at d = 64, over more Q blocks (N = 1100, ragged tail) than

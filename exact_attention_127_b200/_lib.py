@@ -78,6 +78,9 @@ def load_library():
     lib.attn_decode_test_wait_timeout.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, vp,
                                                   ctypes.c_size_t, vp]
     lib.attn_decode_test_wait_timeout.restype = c_int
+    lib.attn_bwd_test_wait_timeout.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64,
+                                               c_int, vp, ctypes.c_size_t, vp]
+    lib.attn_bwd_test_wait_timeout.restype = c_int
     i32p = ctypes.POINTER(ctypes.c_int32)
     lib.attn_fwd_schedule.argtypes = [i64, i64, i64, c_int, c_int, i32p, i32p, i64]
     lib.attn_fwd_schedule.restype = i64

@@ -81,6 +81,7 @@ struct BwdParams {
     float scale;         // multiplies q.k
     float scale_log2;    // scale * log2(e)
     uint64_t wait_limit_ns;
+    int withhold;        // test hook: the TMA warp loads nothing, so every wait runs out
 };
 
 template <int D>
@@ -308,7 +309,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (warp == BWD_LOAD_WARP) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(BWD_CTRL_REGS) : "memory");
         /* ---------------- TMA: K_j, V_j once; Q_i, dO_i per Q block ---------------- */
-        if (lane == 0) {
+        if (lane == 0 && !p.withhold) {
             mbar_arrive_expect_tx(bar_kv, 2 * TILE);
             for (int c = 0; c < C::CHUNKS; ++c) {
                 tma_load_3d(&tm_k, sK + c * CHUNK_BYTES, bar_kv, c * CHUNK_ELEMS, jb * BLOCK_M, bh);

@@ -1689,7 +1689,7 @@ int bwd_launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
 int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
              const float* lse, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N,
              int64_t d, int causal, float scale, void* workspace, size_t workspace_bytes,
-             void* stream) {
+             void* stream, uint64_t wait_limit_ns, int withhold) {
     bool empty = false;
     int st = validate_shape(B, H, N, d, scale, &empty);
     if (st != ATTN_OK || empty) return st;
@@ -1737,7 +1737,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     prm.nblk = static_cast<int>(Np / BLOCK_M);
     prm.scale = scale;
     prm.scale_log2 = scale * LOG2E;
-    prm.wait_limit_ns = WAIT_LIMIT_NS;
+    prm.wait_limit_ns = wait_limit_ns;
+    prm.withhold = withhold;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const auto* ob = static_cast<const __nv_bfloat16*>(o);
     const auto* db = static_cast<const __nv_bfloat16*>(dout);
@@ -1824,7 +1825,15 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
              int64_t d, int causal, float scale, void* workspace, size_t workspace_bytes,
              void* stream) {
     return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, workspace,
-                    workspace_bytes, stream);
+                    workspace_bytes, stream, WAIT_LIMIT_NS, 0);
+}
+
+int attn_bwd_test_wait_timeout(const void* q, const void* k, const void* v, const void* o,
+                               const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                               int64_t B, int64_t H, int64_t N, int64_t d, int causal,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+    return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, causal, 0.125f, workspace,
+                    workspace_bytes, stream, TEST_WAIT_LIMIT_NS, 1);
 }
 
 size_t attn_standard_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {

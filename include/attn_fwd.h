@@ -277,6 +277,20 @@ int attn_decode_test_wait_timeout(const void* q, const void* k, const void* v, v
                                   size_t workspace_bytes, void* stream);
 
 /*
+ * attn_bwd_test_wait_timeout -- the same test hook for the backward pass.
+ * Takes attn_bwd's arguments minus scale, with the same checks.  The pre
+ * kernel runs as usual.  In the main kernel the TMA warp is told to load
+ * nothing (no K, V, Q or dO), and every bounded wait is limited to 20 ms.  The
+ * waits run out and ATTN_ERR_TIMEOUT goes to the device status word.  Every
+ * CTA then frees its tensor memory and exits.  dq, dk, dv and the workspace
+ * are left unspecified.
+ */
+int attn_bwd_test_wait_timeout(const void* q, const void* k, const void* v, const void* o,
+                               const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                               int64_t B, int64_t H, int64_t N, int64_t d, int causal,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * attn_fwd_schedule -- host-only query of the forward kernel's static work
  * schedule (no CUDA call; usable without a GPU).  The work is split into units
  * of two 128-row Q tiles of one head: unit u = bh * ceil(N/256) + pair covers

@@ -1,5 +1,5 @@
-"""Element offsets beyond 2^31: every entry point on tensors of more than 2^31
-elements.
+"""Element offsets beyond 2^31: the forward (bf16 and e4m3), backward and
+decode entry points on tensors of more than 2^31 elements.
 
 B=1, H=8200, N=2048, d=128 makes 2.15e9 elements per [B, H, N, d] tensor, so
 the last heads' elements lie past the range of a 32-bit index (the bf16
@@ -114,3 +114,35 @@ def test_decode_beyond_2_31_elements(lib):
     assert abs(lse[0, MID].item() - math.log(N)) <= 1e-4
     del q, k, v, o, lse
     _release()
+
+
+def test_fp8_forward_beyond_2_31_elements(lib):
+    """e4m3 operands (1 byte per element, so 2.15 GB per tensor, and V^T in the
+    workspace), checked like tests/test_fp8.py: the oracle on the dequantized
+    values, per-element bound (2^-4 + 2^-8) max_j |v_jc| + 1e-3, relative L2
+    below 5 %."""
+    sq, sk, sv = (t[0] for t in inputs.make_qkv_e4m3(1, 2, N, D, seed=65))
+
+    def big8(fill):
+        t = torch.zeros((B, H, N, D), dtype=torch.float8_e4m3fn, device="cuda")
+        for j, h in enumerate(FILLED):
+            t[0, h].copy_(fill[j])
+        return t
+
+    q8, k8, v8 = big8(sq), big8(sk), big8(sv)
+    o, lse = lib.attn_fwd_fp8(q8, k8, v8, causal=True, scale=SCALE)
+    torch.cuda.synchronize()
+    assert lib.device_status(reset=True) == 0
+    rows = inputs.sample_rows(N, 128, 65)
+    qd, kd, vd = (t.to(torch.float64)[None] for t in (sq, sk, sv))
+    O_ref, L_ref = oracle.attention_rows(qd, kd, vd, True, SCALE, rows=rows)
+    of = o[0, list(FILLED)][:, rows].double().cpu().numpy()
+    lf = lse[0, list(FILLED)][:, rows].double().cpu().numpy()
+    vmax = np.maximum.accumulate(np.abs(vd[0].numpy()), axis=1)[:, rows]     # over keys j <= i
+    assert np.all(np.abs(of - O_ref) <= (2.0 ** -4 + 2.0 ** -8) * vmax + 1e-3)
+    assert np.linalg.norm(of - O_ref) / np.linalg.norm(O_ref) <= 5e-2
+    assert np.abs(lf - L_ref).max() <= LSE_MAX_ABS
+    assert not o[0, MID].any()
+    del q8, k8, v8, o, lse
+    _release()
+

@@ -95,6 +95,19 @@ def test_empty_problem_is_ok_without_pointers(lib):
     assert _call(lib, q=None, k=None, v=None, o=None, lse=None, N=0) == OK
 
 
+@pytest.mark.parametrize("B,N", [(0, 100), (1, 0)])
+def test_every_entry_point_accepts_an_empty_problem(lib, B, N):
+    """B * H * N = 0 is a valid problem with nothing to compute: every entry
+    point returns ATTN_OK before it looks at a pointer or the device."""
+    n = None
+    assert lib.attn_fwd_host(n, n, n, n, n, B, 2, N, 64, 1, 0.125, n, 0, n) == OK
+    assert lib.attn_fwd_fp8(n, n, n, 1.0, 1.0, 1.0, n, n, B, 2, N, 128, 1, 0.125, n, 0, n) == OK
+    assert lib.attn_bwd(n, n, n, n, n, n, n, n, n, B, 2, N, 64, 1, 0.125, n, 0, n) == OK
+    assert lib.attn_standard(n, n, n, n, n, B, 2, N, 64, 0, 0.125, n, 0, n) == OK
+    # decode follows the same rule; over N = 0 cached keys it writes nothing
+    assert lib.attn_decode(n, n, n, n, n, B, 2, N, 64, 0.125, n, 0, n) == OK
+
+
 def test_host_entry_point_validation(lib):
     f = lib.attn_fwd_host
     assert lib.attn_fwd_host_workspace_bytes(1, 1, 128, 96) == 0
